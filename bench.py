@@ -1,0 +1,371 @@
+"""Throughput of the hybrid compressed attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Default workload (the one the headline metric is quoted on): one HCA layer prefill, T = 32768
+tokens, bf16, c = 512 (64 RoPE dims), m' = 128 -> 256 compressed entries, 64 query heads,
+window 128, sink.  One step = hca_compress + hybrid_attn_prefill over the whole layer.
+Other workloads (--workload): csa_prefill_64k (csa_compress x2 + indexer_topk +
+hybrid_attn_prefill), csa_decode_1m (indexer_topk FP4 + hybrid_attn_decode over the FP8/BF16
+cache, 8 sequences at position 1,048,576).
+
+Prints ONE JSON line (rank 0).  value = tokens/s of the whole job (all ranks; each rank runs
+its own independent layer: weak scaling, no collective on the data path), measured with CUDA
+events on the launching stream, inputs resident in HBM, max over ranks.  e2e = the same metric
+through the C ABI with the inputs copied from pinned host memory and the output copied back
+inside the timed region.  roofline = the dominant kernel's algorithmic FLOPs per launch / its
+average CUDA-event duration against the measured dense bf16 peak (MEASURED_PEAKS.json).
+cpu_baseline = the fp64 oracle timed on this host's cores on a bounded sample.
+--impl reference times that oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import csa_workloads as WL  # noqa: E402
+
+METRIC = "CSA/HCA attention tokens/s (prefill, 1M-ctx decode) at 1 B200; % of HBM/TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------------------------
+
+def attn_keys_per_token(T: int, W: int, m: int, n_comp: int, k: int | None) -> np.ndarray:
+    t = np.arange(T, dtype=np.int64)
+    win = np.minimum(t + 1, W)
+    vis = np.minimum((t + 1) // m, n_comp)
+    return win + (np.minimum(vis, k) if k is not None else vis)
+
+
+def attn_flops(T, H, c, W, m, n_comp, k=None) -> float:
+    """QK^T and PV: 2 x 2 x H x c flops per (token, key)."""
+    return float(attn_keys_per_token(T, W, m, n_comp, k).sum()) * H * c * 4.0
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads on the GPU
+# ---------------------------------------------------------------------------------------------
+
+def _to_dev_bf16(x32: np.ndarray, torch, device):
+    return torch.from_numpy(np.ascontiguousarray(x32, np.float32)).to(torch.bfloat16).to(device)
+
+
+def gen_rows_bf16(w, name, rows, ncols, torch, out, seq=0, chunk=2048):
+    """Fill device tensor `out` [rows, ncols] (bf16) with the seeded draws chunk by chunk."""
+    for r0 in range(0, rows, chunk):
+        r1 = min(rows, r0 + chunk)
+        x = WL.draw(w, name, r0, r1, seq=seq)
+        out[r0:r1].copy_(torch.from_numpy(x).to(torch.bfloat16))
+
+
+class HcaPrefill:
+    """One HCA layer prefill: hca_compress (C, Z -> 256 entries) + hybrid_attn_prefill."""
+
+    def __init__(self, w, rank, torch, C, device):
+        self.w, self.torch, self.C, self.dev = w, torch, C, device
+        T, c, H, m = w.T, w.c, w.H, w.m
+        bf = torch.bfloat16
+        self.Cc = torch.empty((T, c), dtype=bf, device=device)
+        self.Z = torch.empty((T, c), dtype=bf, device=device)
+        self.X = torch.empty((T, c), dtype=bf, device=device)
+        self.q = torch.empty((T, H, c), dtype=bf, device=device)
+        for name, t in (("C", self.Cc), ("Z", self.Z), ("X", self.X)):
+            gen_rows_bf16(w, name, T, c, torch, t, seq=rank)
+        gen_rows_bf16(w, "q", T, H * c, torch, self.q.view(T, H * c), seq=rank, chunk=256)
+        self.B = torch.from_numpy(WL.normal_rows(w.seed, f"B/L0/S{rank}", c, 0, m, std=w.bias_std)).to(device)
+        self.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, seq=rank)[0]).to(device)
+        self.kv = torch.empty((T // m, c), dtype=bf, device=device)
+        self.o = torch.empty_like(self.q)
+        self.scale = 1.0
+        self.flops = attn_flops(T, H, c, w.W, m, T // m)
+        self.tokens = T
+        self.launches_per_step = 2
+
+    def step(self, ev=None):
+        C = self.C
+        C.hca_compress(self.Cc, self.Z, self.B, self.w.m, out=self.kv)
+        if ev is not None:
+            ev[0].record()
+        C.hybrid_attn_prefill(self.q, self.X, self.kv, self.sink, self.scale, self.w.m, self.w.W, o=self.o)
+        if ev is not None:
+            ev[1].record()
+
+    # end-to-end through the C ABI: pinned host inputs -> device -> compute -> host output
+    def setup_e2e(self):
+        torch = self.torch
+        self.h_in = [t.cpu().pin_memory() for t in (self.Cc, self.Z, self.X, self.q)]
+        self.h_out = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in) + self.B.numel() * 4 + self.sink.numel() * 4
+        self.d2h = self.o.numel() * self.o.element_size()
+        self.h_small = [self.B.cpu().pin_memory(), self.sink.cpu().pin_memory()]
+
+    def step_e2e(self):
+        for d, h in zip((self.Cc, self.Z, self.X, self.q), self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.B.copy_(self.h_small[0], non_blocking=True)
+        self.sink.copy_(self.h_small[1], non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.o, non_blocking=True)
+
+
+WORKLOADS = {"hca_prefill_32k": HcaPrefill}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------------------------
+
+def oracle_hca_sample(w, n_tokens: int, seed_rank: int = 0):
+    """Time the oracle on a bounded sample of the HCA layer: the full compression (amortised
+    over T) plus attention of n_tokens query tokens spread over the sequence.
+    Returns (tokens/s, seconds, description)."""
+    import oracle as O
+    T, c, H, m, W = w.T, w.c, w.H, w.m, w.W
+    Cc = WL.draw(w, "C", 0, T, seq=seed_rank)
+    Z = WL.draw(w, "Z", 0, T, seq=seed_rank)
+    B = WL.normal_rows(w.seed, f"B/L0/S{seed_rank}", c, 0, m, std=w.bias_std)
+    rows = np.linspace(0, T - 1, n_tokens).astype(np.int64)
+    qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1, seq=seed_rank)[0] for t in rows]).reshape(n_tokens, H, c)
+    X = WL.draw(w, "X", 0, T, seq=seed_rank)
+    sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
+    t0 = time.perf_counter()
+    KV = O.hca_compress(Cc, Z, B, m)
+    t1 = time.perf_counter()
+    O.hybrid_attn_prefill(qs, X, KV, sink, 1.0, m, W, rows=rows)
+    t2 = time.perf_counter()
+    per_token = (t1 - t0) / T + (t2 - t1) / n_tokens
+    desc = (f"full hca_compress of T={T} (amortised per token) + hybrid attention of {n_tokens} query tokens "
+            f"evenly spaced over the layer")
+    return 1.0 / per_token, (t2 - t0), desc
+
+
+# ---------------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="hca_prefill_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = WL.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, w, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", init_method="env://", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    import compressed_sparse_kv_csa_b200 as C
+
+    job = WORKLOADS[args.workload](w, rank, torch, C, device)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(args.warmup, 3)):
+        job.step()
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            job.step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(stop) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    t = torch.tensor([ms, kern_ms], device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, kern_ms = float(t[0]), float(t[1])
+
+    # end to end through the C ABI with host buffers
+    job.setup_e2e()
+    job.step_e2e()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        job.step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    te = torch.tensor([e2e_ms], device=device)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(te[0])
+
+    if rank == 0:
+        pk, src = peaks()
+        achieved = job.flops / (kern_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC,
+            "value": world * job.tokens / (ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": max(args.warmup, 3),
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs on the bf16 grid, no trained weights)",
+            "config": {"workload": args.workload, "T": w.T, "c": w.c, "rope_dims": w.rope, "m": w.m, "H": w.H,
+                       "W": w.W, "n_comp": w.T // w.m, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (q alone is 2.1 GB)"},
+            "roofline": {"bound": "tensor", "kernel": "hybrid_attn_prefill", "achieved": achieved,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                         "peak_source": f"{src} dense bf16 burst", "traffic": None,
+                         "flops_per_launch": job.flops, "launch_ms": kern_ms},
+            "e2e": {"value": world * job.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": job.h2d, "d2h_bytes_per_step": job.d2h, "ms_per_step": e2e_ms},
+            "clocks": clk.summary(),
+            "gpu_launches": job.launches_per_step * args.steps,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            import oracle as O
+            tps, secs, desc = oracle_hca_sample(w, 16)
+            n = int(min(4096, max(16, 12.0 / max(secs, 1e-3) * 16)))
+            tps, secs, desc = oracle_hca_sample(w, n)
+            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
+                                    "sample": desc, "seconds": secs}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference_arm(args, w, world, rank):
+    """The fp64 oracle as the reference implementation, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle as O
+    n = 64
+    for _ in range(max(args.warmup, 3)):
+        oracle_hca_sample(w, n)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        tps, s, desc = oracle_hca_sample(w, n)
+        vals.append(tps)
+        secs.append(s)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "T": w.T, "c": w.c, "m": w.m, "H": w.H, "W": w.W},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

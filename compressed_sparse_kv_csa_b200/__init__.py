@@ -1,0 +1,295 @@
+"""compressed_sparse_kv_csa_b200 -- the hybrid compressed attention hot path of DeepSeek-V4
+(CSA / HCA compression, lightning-indexer top-k, hybrid MQA attention with sink) as hand-written
+CUDA for sm_100a, behind the C ABI declared in include/csa.h.
+
+This module is a thin binding with the same names as the C entry points: it only marshals
+torch tensors (device memory, streams) into pointers and sizes.  Every step of the path runs in
+libcsa.so; if the library is missing the import fails, and there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK = 0
+CSA_ERR_INVALID_ARG = -1
+CSA_ERR_UNSUPPORTED = -2
+CSA_ERR_CUDA = -3
+CSA_ERR_WORKSPACE = -5
+CSA_DEVERR_TIMEOUT = 1
+CSA_DEVERR_INDEX = 2
+CSA_F32 = 0
+CSA_BF16 = 1
+CSA_FP4 = 2
+
+EXPORTED = ("csa_compress", "hca_compress", "csa_quantize_kv", "csa_quantize_fp4",
+            "indexer_topk_workspace_size", "indexer_topk", "hybrid_attn_prefill",
+            "hybrid_attn_decode_workspace_size", "hybrid_attn_decode", "csa_device_error",
+            "csa_status_string", "csa_abi_version")
+
+
+class CsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        self.status = status
+
+
+class _KvRows(ctypes.Structure):
+    _fields_ = [("fp8", ctypes.c_void_p), ("rope", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("c", ctypes.c_int32), ("rope_dims", ctypes.c_int32)]
+
+
+class _Fp4Rows(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("n", ctypes.c_int64),
+                ("d", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libcsa.so not found at {LIB_PATH}: build it with "
+                          "`python -m compressed_sparse_kv_csa_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    P_kv, P_f4 = ctypes.POINTER(_KvRows), ctypes.POINTER(_Fp4Rows)
+    sig = {
+        "csa_compress": ([vp, vp, vp, vp, vp, i64, i32, i32, i32, vp, i32, P_kv, P_f4, vp], ctypes.c_int),
+        "hca_compress": ([vp, vp, vp, i64, i32, i32, i32, vp, i32, P_kv, vp], ctypes.c_int),
+        "csa_quantize_kv": ([vp, i32, i64, i32, i32, P_kv, vp], ctypes.c_int),
+        "csa_quantize_fp4": ([vp, i32, i64, i32, P_f4, vp], ctypes.c_int),
+        "indexer_topk_workspace_size": ([i64, i64, i32], sz),
+        "indexer_topk": ([vp, vp, vp, i32, vp, vp, i64, i64, i32, i32, i32, i32, i64, vp, vp, vp, sz, vp],
+                         ctypes.c_int),
+        "hybrid_attn_prefill": ([vp, vp, vp, i64, vp, i32, vp, f32, i64, i32, i32, i32, i32, i32, vp, vp, vp],
+                                ctypes.c_int),
+        "hybrid_attn_decode_workspace_size": ([i32, i32, i32, i32, i32, i64, i32], sz),
+        "hybrid_attn_decode": ([vp, P_kv, vp, vp, P_kv, vp, vp, i32, vp, f32, i32, i32, i32, i32, i32, i64,
+                                vp, vp, vp, sz, vp], ctypes.c_int),
+        "csa_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
+        "csa_status_string": ([i32], ctypes.c_char_p),
+        "csa_abi_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.csa_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != CSA_OK:
+        raise CsaError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        if torch.cuda.is_available():
+            return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        return None
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return CSA_F32
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ----------------------------------------------------------------------------------------
+# cache containers (torch owns the memory)
+# ----------------------------------------------------------------------------------------
+
+@dataclass
+class KvRows:
+    """Mixed-precision KV rows: fp8 [n, c-rope] uint8, rope [n, rope] bf16, scale [n] fp32."""
+    fp8: torch.Tensor
+    rope: torch.Tensor
+    scale: torch.Tensor
+
+    @property
+    def n(self) -> int:
+        return self.fp8.shape[0]
+
+    @property
+    def c(self) -> int:
+        return self.fp8.shape[1] + self.rope.shape[1]
+
+    @property
+    def rope_dims(self) -> int:
+        return self.rope.shape[1]
+
+    @staticmethod
+    def empty(n: int, c: int, rope_dims: int, device) -> "KvRows":
+        return KvRows(torch.empty((n, c - rope_dims), dtype=torch.uint8, device=device),
+                      torch.empty((n, rope_dims), dtype=torch.bfloat16, device=device),
+                      torch.empty((n,), dtype=torch.float32, device=device))
+
+    def _c(self) -> _KvRows:
+        return _KvRows(self.fp8.data_ptr(), self.rope.data_ptr() if self.rope.numel() else 0,
+                       self.scale.data_ptr(), self.n, self.c, self.rope_dims)
+
+
+@dataclass
+class Fp4Rows:
+    """FP4 E2M1 rows: codes [n, d/2] uint8 (element 2i in the low nibble), scales [n, d/32] E8M0."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+
+    @property
+    def n(self) -> int:
+        return self.codes.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.codes.shape[1] * 2
+
+    @staticmethod
+    def empty(n: int, d: int, device) -> "Fp4Rows":
+        return Fp4Rows(torch.empty((n, d // 2), dtype=torch.uint8, device=device),
+                       torch.empty((n, d // 32), dtype=torch.uint8, device=device))
+
+    def _c(self) -> _Fp4Rows:
+        return _Fp4Rows(self.codes.data_ptr(), self.scales.data_ptr(), self.n, self.d)
+
+
+# ----------------------------------------------------------------------------------------
+# entry points
+# ----------------------------------------------------------------------------------------
+
+def csa_compress(Ca, Cb, Za, Zb, B, m: int, out=None, out_kv: KvRows | None = None,
+                 out_fp4: Fp4Rows | None = None, stream=None):
+    """Overlapped CSA compression into ``out`` [T//m, c] (fp32/bf16) and/or the caches."""
+    T, c = Ca.shape
+    st = _lib.csa_compress(_ptr(Ca), _ptr(Cb), _ptr(Za), _ptr(Zb), _ptr(B), T, c, m, _dtype_code(Ca),
+                           _ptr(out), _dtype_code(out) if out is not None else 0,
+                           ctypes.byref(out_kv._c()) if out_kv is not None else None,
+                           ctypes.byref(out_fp4._c()) if out_fp4 is not None else None, _stream(stream))
+    _check("csa_compress", st)
+    return out
+
+
+def hca_compress(C, Z, B, m: int, out=None, out_kv: KvRows | None = None, stream=None):
+    """HCA compression into ``out`` [T//m, c] and/or the mixed KV cache."""
+    T, c = C.shape
+    st = _lib.hca_compress(_ptr(C), _ptr(Z), _ptr(B), T, c, m, _dtype_code(C), _ptr(out),
+                           _dtype_code(out) if out is not None else 0,
+                           ctypes.byref(out_kv._c()) if out_kv is not None else None, _stream(stream))
+    _check("hca_compress", st)
+    return out
+
+
+def csa_quantize_kv(x, out: KvRows, stream=None):
+    n, c = x.shape
+    _check("csa_quantize_kv", _lib.csa_quantize_kv(_ptr(x), _dtype_code(x), n, c, out.rope_dims,
+                                                   ctypes.byref(out._c()), _stream(stream)))
+    return out
+
+
+def csa_quantize_fp4(x, out: Fp4Rows, stream=None):
+    n, d = x.shape
+    _check("csa_quantize_fp4", _lib.csa_quantize_fp4(_ptr(x), _dtype_code(x), n, d, ctypes.byref(out._c()),
+                                                     _stream(stream)))
+    return out
+
+
+def indexer_topk_workspace_size(Nq: int, max_nvis: int, k: int) -> int:
+    return int(_lib.indexer_topk_workspace_size(Nq, max_nvis, k))
+
+
+def indexer_topk(q, w, keys, m: int, k: int, max_nvis: int, q_pos=None, key_off=None, n_keys=None,
+                 H_I=None, d_I=None, idx_out=None, score_out=None, workspace=None, stream=None):
+    """Indexer scores + top-k.  Dense: q [Nq,H_I,d_I], keys [n_keys,d_I] (fp32/bf16).
+    FP4: q and keys are Fp4Rows (q rows = Nq*H_I).  Returns idx_out [Nq, k] int32."""
+    if isinstance(q, Fp4Rows):
+        fmt = CSA_FP4
+        Nq = w.shape[0]
+        H_I = w.shape[1]
+        d_I = q.d
+        n_keys = keys.n if n_keys is None else n_keys
+        qarg, karg = ctypes.byref(q._c()), ctypes.byref(keys._c())
+        device = q.codes.device
+    else:
+        fmt = _dtype_code(q)
+        Nq, H_I, d_I = q.shape
+        n_keys = keys.shape[0] if n_keys is None else n_keys
+        qarg, karg = _ptr(q), _ptr(keys)
+        device = q.device
+    if idx_out is None:
+        idx_out = torch.empty((Nq, k), dtype=torch.int32, device=device)
+    need = indexer_topk_workspace_size(Nq, max_nvis, k)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=device)
+    st = _lib.indexer_topk(qarg, _ptr(w), karg, fmt, _ptr(q_pos), _ptr(key_off), n_keys, Nq, H_I, d_I, m, k,
+                           max_nvis, _ptr(idx_out), _ptr(score_out), _ptr(workspace), workspace.numel(),
+                           _stream(stream))
+    _check("indexer_topk", st)
+    return idx_out
+
+
+def hybrid_attn_prefill(q, x_win, kv_comp, sink, scale: float, m: int, W: int, idx=None, o=None,
+                        lse=None, stream=None):
+    """Hybrid MQA attention for prefill; q [T,H,c], x_win [T,c], kv_comp [n_comp,c]."""
+    T, H, c = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    k = idx.shape[1] if idx is not None else 0
+    st = _lib.hybrid_attn_prefill(_ptr(q), _ptr(x_win), _ptr(kv_comp), kv_comp.shape[0], _ptr(idx), k,
+                                  _ptr(sink), float(scale), T, H, c, m, W, _dtype_code(q), _ptr(o), _ptr(lse),
+                                  _stream(stream))
+    _check("hybrid_attn_prefill", st)
+    return o
+
+
+def hybrid_attn_decode_workspace_size(B: int, H: int, c: int, k: int, W: int, max_nvis: int,
+                                      use_idx: bool) -> int:
+    return int(_lib.hybrid_attn_decode_workspace_size(B, H, c, k, W, max_nvis, int(use_idx)))
+
+
+def hybrid_attn_decode(q, comp: KvRows, comp_off, pos, win: KvRows, win_len, sink, scale: float, m: int,
+                       W: int, max_nvis: int, idx=None, o=None, lse=None, workspace=None, stream=None):
+    """Hybrid attention for one new token per sequence over the mixed FP8/BF16 caches."""
+    B, H, c = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    k = idx.shape[1] if idx is not None else 0
+    need = hybrid_attn_decode_workspace_size(B, H, c, k, W, max_nvis, idx is not None)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
+    st = _lib.hybrid_attn_decode(_ptr(q), ctypes.byref(comp._c()), _ptr(comp_off), _ptr(pos),
+                                 ctypes.byref(win._c()), _ptr(win_len), _ptr(idx), k, _ptr(sink), float(scale),
+                                 B, H, c, m, W, max_nvis, _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                 _stream(stream))
+    _check("hybrid_attn_decode", st)
+    return o
+
+
+def csa_device_error(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("csa_device_error", _lib.csa_device_error(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
+
+
+def csa_abi_version() -> int:
+    return int(_lib.csa_abi_version())

@@ -1,0 +1,153 @@
+// topk.cu -- per-query top-k selection over the indexer scores.
+//
+// Method: "DeepSeek-V4: Towards Highly Efficient Million-Token Context Intelligence" paper notes,
+// Sec. 2.3 Indexer listing: the k_eff = min(k, N_vis) best entries per query.  Ordering
+// convention of this library: score descending, equal scores by lower entry index; unused slots
+// hold -1.
+//
+// One CTA per query row.  Radix select over order-preserving 32-bit keys of the fp32 scores
+// (four 8-bit digit passes with a shared-memory histogram) finds the exact k-th key; entries
+// above it are taken unordered, entries equal to it are taken in index order by a block-wide
+// ordered scan, and the k_eff winners are then sorted in shared memory (bitonic, 64-bit keys
+// (score key, inverted index)).
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int TK_THREADS = 1024;
+constexpr int TK_MAX = 2048;
+
+__device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
+{
+    const int64_t t = a.q_pos ? a.q_pos[r] : r;
+    int64_t nv = (t + 1) / a.m;
+    if (nv > a.max_nvis) nv = a.max_nvis;
+    const int64_t base = a.key_off ? a.key_off[r] : 0;
+    if (base < 0) return 0;
+    if (nv > a.n_keys - base) nv = a.n_keys - base;
+    return nv < 0 ? 0 : nv;
+}
+
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
+{
+    __shared__ unsigned long long sel[TK_MAX];
+    __shared__ int hist[256];
+    __shared__ int s_bin, s_rem, s_cnt, s_warp[TK_THREADS / 32], s_eq_taken;
+    __shared__ uint32_t s_prefix;
+
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t nv = tk_nvis(a, r);
+    const int k = a.k;
+    const int ke = (int)(nv < k ? nv : k);
+    const float *S = a.scores + r * a.ld;
+
+    uint32_t thr = 0;   // k-th largest key (only meaningful when nv > k)
+    int n_gt = 0;       // number of keys strictly above thr
+    if (nv > k) {
+        uint32_t prefix = 0, pmask = 0;
+        int rem = k;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0;
+            __syncthreads();
+            for (int64_t s = tid; s < nv; s += TK_THREADS) {
+                const uint32_t key = float_key(S[s]);
+                if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int cum = 0, b = 255;
+                for (; b > 0; --b) {
+                    if (cum + hist[b] >= rem) break;
+                    cum += hist[b];
+                }
+                s_bin = b;
+                s_rem = rem - cum;
+            }
+            __syncthreads();
+            prefix |= uint32_t(s_bin) << shift;
+            pmask |= 255u << shift;
+            rem = s_rem;
+            __syncthreads();
+        }
+        thr = prefix;
+        n_gt = k - rem;
+        if (tid == 0) { s_cnt = 0; s_prefix = thr; s_eq_taken = 0; }
+        __syncthreads();
+        // strictly greater: unordered append
+        for (int64_t s = tid; s < nv; s += TK_THREADS) {
+            const uint32_t key = float_key(S[s]);
+            if (key > thr) {
+                const int pos = atomicAdd(&s_cnt, 1);
+                if (pos < n_gt) sel[pos] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)s);
+            }
+        }
+        __syncthreads();
+        // equal to the threshold: the lowest indices first (ordered block scan)
+        const int need = rem;
+        for (int64_t base = 0; base < nv; base += TK_THREADS) {
+            if (s_eq_taken >= need) break; // uniform: read after a barrier
+            const int64_t s = base + tid;
+            const bool eq = (s < nv) && (float_key(S[s]) == thr);
+            const unsigned bal = __ballot_sync(0xffffffffu, eq);
+            const int lane = tid & 31, wid = tid >> 5;
+            if (lane == 0) s_warp[wid] = __popc(bal);
+            __syncthreads();
+            int before = 0, total = 0;
+            for (int w = 0; w < TK_THREADS / 32; ++w) {
+                if (w < wid) before += s_warp[w];
+                total += s_warp[w];
+            }
+            const int rank = s_eq_taken + before + __popc(bal & ((1u << lane) - 1u));
+            if (eq && rank < need) sel[n_gt + rank] = ((unsigned long long)thr << 32) | (0xffffffffu - (uint32_t)s);
+            __syncthreads();
+            if (tid == 0) s_eq_taken += total;
+            __syncthreads();
+        }
+    } else {
+        for (int64_t s = tid; s < nv; s += TK_THREADS)
+            sel[s] = ((unsigned long long)float_key(S[s]) << 32) | (0xffffffffu - (uint32_t)s);
+    }
+    // bitonic sort (descending) of the ke winners, padded with zeros to a power of two
+    int n2 = 1;
+    while (n2 < ke) n2 <<= 1;
+    for (int i = ke + tid; i < n2; i += TK_THREADS) sel[i] = 0ull;
+    __syncthreads();
+    for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < n2; i += TK_THREADS) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool desc = (i & size) == 0;
+                    const unsigned long long x = sel[i], y = sel[j];
+                    if (desc ? (x < y) : (x > y)) { sel[i] = y; sel[j] = x; }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int j = tid; j < k; j += TK_THREADS) {
+        int32_t id = -1;
+        float sc = -INFINITY;
+        if (j < ke) {
+            const unsigned long long v = sel[j];
+            id = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffu));
+            sc = key_float((uint32_t)(v >> 32));
+        }
+        a.idx_out[r * k + j] = id;
+        if (a.score_out) a.score_out[r * k + j] = sc;
+    }
+}
+
+} // namespace
+
+cudaError_t launch_topk(const IndexerArgs &a, cudaStream_t st)
+{
+    if (a.Nq == 0) return cudaSuccess;
+    topk_kernel<<<(unsigned)a.Nq, TK_THREADS, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+} // namespace csa

@@ -194,3 +194,19 @@ def mixed_lengths(w: Workload) -> np.ndarray:
     lo, hi = w.extra["len_lo"], w.extra["len_hi"]
     u = g.random(w.B)
     return np.floor(np.exp(np.log(lo) + u * (np.log(hi) - np.log(lo)))).astype(np.int64)
+
+
+def random_topk_idx(seed: int, T: int, m: int, k: int, n_comp: int, rows=None) -> np.ndarray:
+    """A synthetic top-k index list per query (attention-only parity): for query t, k distinct
+    entries drawn uniformly from the visible ones s < min(floor((t+1)/m), n_comp), -1 padded
+    when fewer are visible.  Row t is drawn from its own seeded stream."""
+    rows = range(T) if rows is None else rows
+    out = np.full((len(rows), k), -1, dtype=np.int32)
+    for i, t in enumerate(rows):
+        nv = min((int(t) + 1) // m, n_comp)
+        if nv == 0:
+            continue
+        g = rng(seed, "topk_idx", int(t))
+        n = min(k, nv)
+        out[i, :n] = g.choice(nv, size=n, replace=False)
+    return out

@@ -1,0 +1,230 @@
+/*
+ * csa.h -- C ABI of libcsa: the hybrid compressed attention hot path of DeepSeek-V4 (CSA / HCA)
+ * as hand-written CUDA for sm_100a (B200).
+ *
+ * Sources (page title and section):
+ *   [notes]  "DeepSeek-V4: Towards Highly Efficient Million-Token Context Intelligence" paper
+ *            notes (jimmysue.github.io), Sec. 2.3 CSA (Eq. 11-12, Eq. 16, Compressor and Indexer
+ *            listings) and Sec. 2.4 HCA (Eq. 22-23, Attention.forward listing).
+ *   [qa]     itsolotime.com Q&A essay on DeepSeek-V4, Question 1 (sliding window, overlapped
+ *            compression, attention sink) and Question 4 (FP4 E2M1, FP8 E4M3).
+ *   [ledger] "Mind Observatory: Uncovering the technical ledger of DeepSeek-V4" (RoPE dims of the
+ *            KV cache in BF16, the rest in FP8; indexer QK path in FP4).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless stated otherwise.  The
+ *     library allocates nothing; scratch comes from a caller-provided workspace whose size is
+ *     returned by the matching *_workspace_size() call.
+ *   - Arrays are row-major and densely packed.  T = tokens, c = KV channels, m = compression
+ *     ratio, H = query heads, H_I / d_I = index heads / index head dim, W = window, k = top-k.
+ *   - N_vis(t) = floor((t+1)/m) is the number of compressed entries visible to the query at
+ *     0-based position t: an entry becomes visible once its last token is at or before t, so a
+ *     query never sees the block it is still inside.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only enqueue work and
+ *     return immediately; results are ready when the stream reaches them.
+ *   - Return value: CSA_OK, or a negative status.  Argument checks run on the host before any
+ *     work is enqueued, so an error return means nothing was launched.  CSA_ERR_CUDA means a
+ *     launch failed (the CUDA error is left for cudaGetLastError()).  Kernels never trap: a
+ *     bounded wait that runs out, or an index the kernel refuses to follow, sets a device error
+ *     word that csa_device_error() reads back.
+ *   - dtype codes: CSA_F32 (fp32) and CSA_BF16 (bf16, stored as uint16 bit patterns).
+ *   - Numerics: inputs bf16 / fp32 / fp8 / fp4, all accumulation and softmax in fp32.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA_OK 0
+#define CSA_ERR_INVALID_ARG (-1)   /* null pointer, bad size, unsupported combination */
+#define CSA_ERR_UNSUPPORTED (-2)   /* valid request with no kernel instance (e.g. c % 32 != 0) */
+#define CSA_ERR_CUDA (-3)          /* a kernel launch failed */
+#define CSA_ERR_WORKSPACE (-5)     /* workspace missing or smaller than *_workspace_size() */
+
+/* device error word bits (csa_device_error) */
+#define CSA_DEVERR_TIMEOUT 1       /* a bounded wait ran out */
+#define CSA_DEVERR_INDEX 2         /* an out-of-range index was skipped */
+
+#define CSA_F32 0
+#define CSA_BF16 1
+#define CSA_FP4 2                  /* indexer only: q and keys given as csa_fp4_rows */
+
+/*
+ * Mixed-precision KV rows ([ledger]): the last `rope_dims` channels of each row (the RoPE dims;
+ * the Indexer listing of [notes] rotates q[..., -rd:]) are kept as bf16, the first
+ * c - rope_dims channels as FP8 E4M3 (OCP "fn" variant, max 448) with one fp32 scale per row:
+ *   value[j] = e4m3(fp8[r, j]) * scale[r]        for j <  c - rope_dims
+ *   value[j] = bf16(rope[r, j - (c-rope_dims)])  for j >= c - rope_dims
+ * Planes: fp8 [n, c-rope_dims] bytes, rope [n, rope_dims] bf16 bits, scale [n] fp32.
+ * Each plane base must be 16-byte aligned and (c - rope_dims) and rope_dims multiples of 16.
+ */
+typedef struct csa_kv_rows {
+    uint8_t *fp8;
+    uint16_t *rope;
+    float *scale;
+    int64_t n;
+    int32_t c;
+    int32_t rope_dims;
+} csa_kv_rows;
+
+/*
+ * FP4 rows ([qa] Question 4, [ledger]): E2M1 elements with one E8M0 scale per 32 consecutive
+ * elements (OCP MX v1.0 layout): value[j] = e2m1(nibble j) * 2^(scales[r, j/32] - 127).
+ * codes [n, d/2] bytes (element 2i in the low nibble of byte i), scales [n, d/32] bytes.
+ * d must be a multiple of 32; bases 16-byte aligned.
+ */
+typedef struct csa_fp4_rows {
+    uint8_t *codes;
+    uint8_t *scales;
+    int64_t n;
+    int32_t d;
+} csa_fp4_rows;
+
+/* ----------------------------------------------------------------------------------------- */
+
+/*
+ * csa_compress -- overlapped token-level compression of a CSA layer ([notes] Sec. 2.3,
+ * Eq. 11-12 and the Compressor listing; [qa] Question 1 mechanism 2).
+ *
+ * Entry i (0 <= i < floor(T/m)) pools, per channel d, 2m candidates under ONE softmax:
+ *   current block  p = i*m+j:     value Ca[p,d], logit Za[p,d] + B[j,d]
+ *   previous block p = (i-1)*m+j: value Cb[p,d], logit Zb[p,d] + B[m+j,d]   (only for i >= 1)
+ * so entry 0 pools only its own m tokens, and a trailing partial block is not emitted.
+ *
+ *   Ca, Cb, Za, Zb  [T, c] in `in_dtype` (CSA_F32 or CSA_BF16)
+ *   B               [2m, c] fp32: rows 0..m-1 = B^a (current block), rows m..2m-1 = B^b
+ *   T >= 0, 1 <= m <= 64, c a multiple of 4 and <= 2048
+ * Outputs (any subset, at least one non-NULL):
+ *   out      [floor(T/m), c] in `out_dtype` (CSA_F32 or CSA_BF16)
+ *   out_kv   mixed FP8/BF16 rows (quantise-on-write), out_kv->n >= floor(T/m), ->c == c
+ *   out_fp4  FP4 rows (quantise-on-write, for index keys), ->n >= floor(T/m), ->d == c
+ * Errors: CSA_ERR_INVALID_ARG for null inputs, m out of range, c not supported, or a cache
+ * whose shape does not match.
+ */
+int csa_compress(const void *Ca, const void *Cb, const void *Za, const void *Zb, const float *B,
+                 int64_t T, int32_t c, int32_t m, int32_t in_dtype, void *out, int32_t out_dtype,
+                 const csa_kv_rows *out_kv, const csa_fp4_rows *out_fp4, void *stream);
+
+/*
+ * hca_compress -- heavy compression of an HCA layer ([notes] Sec. 2.4, Eq. 22-23): entry i is
+ * the per-channel softmax pooling of tokens i*m .. i*m+m-1 with logits Z[p,d] + B[p-i*m,d].
+ * No overlap; a trailing partial block is not emitted.
+ *   C, Z [T, c] in `in_dtype`;  B [m, c] fp32;  1 <= m <= 1024.
+ * Outputs as for csa_compress (out, out_kv; at least one non-NULL).
+ */
+int hca_compress(const void *C, const void *Z, const float *B, int64_t T, int32_t c, int32_t m,
+                 int32_t in_dtype, void *out, int32_t out_dtype, const csa_kv_rows *out_kv,
+                 void *stream);
+
+/*
+ * csa_quantize_kv -- write rows x [n, c] (`in_dtype`) into the mixed FP8/BF16 layout of
+ * csa_kv_rows ([ledger]).  Per row: s = amax(|x[0:c-rope]|) / 448 (fp32 division; s = 1 when
+ * that is not positive), fp8 = e4m3(x / s) rounded to nearest even and saturated at 448,
+ * rope = bf16(x[c-rope:c]) rounded to nearest even.
+ */
+int csa_quantize_kv(const void *x, int32_t in_dtype, int64_t n, int32_t c, int32_t rope_dims,
+                    const csa_kv_rows *out, void *stream);
+
+/*
+ * csa_quantize_fp4 -- write rows x [n, d] (`in_dtype`) as FP4 rows.  Per block of 32: the scale
+ * exponent is the smallest e with amax <= 6 * 2^e (clamped to [-127, 127]; -127 for an all-zero
+ * block), element = e2m1(x / 2^e) rounded to nearest even, every zero encoded as +0.
+ */
+int csa_quantize_fp4(const void *x, int32_t in_dtype, int64_t n, int32_t d,
+                     const csa_fp4_rows *out, void *stream);
+
+/* ----------------------------------------------------------------------------------------- */
+
+/*
+ * indexer_topk -- lightning-indexer scores and per-query top-k ([notes] Sec. 2.3, Eq. 16 and
+ * the Indexer listing):
+ *   I[r, s] = sum_h w[r,h] * max(0, q[r,h,:] . K[key_off[r] + s, :])   for s < nv(r)
+ *   nv(r)   = min(floor((q_pos[r]+1)/m), max_nvis, n_keys - key_off[r])
+ * and idx_out[r, :] = the k_eff = min(k, nv(r)) entry indices s with the largest I[r, s],
+ * ordered by score descending, equal scores by lower index; slots k_eff..k-1 hold -1.
+ * One d_I-dim key per compressed entry is shared by all H_I index heads.
+ *
+ *   fmt = CSA_F32 / CSA_BF16: q [Nq, H_I, d_I] and keys [n_keys, d_I] dense in that dtype.
+ *   fmt = CSA_FP4: q is a `const csa_fp4_rows*` with Nq*H_I rows of d_I (row r*H_I + h), keys
+ *                  a `const csa_fp4_rows*` with n_keys rows of d_I.
+ *   w        [Nq, H_I] fp32 head weights (any scaling already folded in by the caller)
+ *   q_pos    [Nq] int64 absolute 0-based positions, or NULL for q_pos[r] = r (prefill)
+ *   key_off  [Nq] int64 first key row of each query's sequence, or NULL for all 0
+ *   max_nvis host-side upper bound of nv(r) (sizes the score buffer)
+ *   idx_out  [Nq, k] int32;  score_out [Nq, k] fp32 scores of the selected entries (or NULL;
+ *            -inf in padded slots)
+ *   ws       workspace of at least indexer_topk_workspace_size(Nq, max_nvis, k) bytes
+ * Limits: 1 <= k <= 2048, 1 <= H_I <= 128, d_I a multiple of 32 (FP4) or 8 and <= 512.
+ */
+size_t indexer_topk_workspace_size(int64_t Nq, int64_t max_nvis, int32_t k);
+int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
+                 const int64_t *q_pos, const int64_t *key_off, int64_t n_keys, int64_t Nq,
+                 int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis,
+                 int32_t *idx_out, float *score_out, void *ws, size_t ws_bytes, void *stream);
+
+/* ----------------------------------------------------------------------------------------- */
+
+/*
+ * hybrid_attn_prefill -- shared-KV multi-query attention of T query tokens over the union of
+ * an uncompressed sliding window and compressed entries, with a per-head sink ([notes]
+ * Sec. 2.3 step 3 and Sec. 2.4 Attention.forward listing; [qa] Question 1 mechanisms 1, 3).
+ * For query t and head h the keys are, concatenated with no de-duplication:
+ *   window:     x_win[u] for u in [max(0, t-W+1), t]      (raw KV rows, the token itself included)
+ *   compressed: kv_comp[s] for s in idx[t, :] with s >= 0  (CSA: the indexer's top-k), or for
+ *               every s < min(N_vis(t), n_comp) when idx is NULL (HCA: all visible entries)
+ * and, with z = scale * q[t,h,:] . key (the key vector is also the value vector),
+ *   o[t,h,:] = sum e^z key / (e^{sink[h]} + sum e^z),  lse[t,h] = ln(e^{sink[h]} + sum e^z).
+ *
+ *   q [T, H, c], x_win [T, c], kv_comp [n_comp, c] in `dtype` (CSA_F32 / CSA_BF16)
+ *   idx [T, k] int32 or NULL; entries outside [0, n_comp) are skipped (CSA_DEVERR_INDEX)
+ *   sink [H] fp32 (-inf allowed: no sink);  o [T, H, c] in `dtype`;  lse [T, H] fp32 or NULL
+ * Limits: c a multiple of 32 and <= 512, 1 <= H <= 128, 1 <= W <= 1024, k <= 4096.
+ */
+int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, int64_t n_comp,
+                        const int32_t *idx, int32_t k, const float *sink, float scale, int64_t T,
+                        int32_t H, int32_t c, int32_t m, int32_t W, int32_t dtype, void *o,
+                        float *lse, void *stream);
+
+/*
+ * hybrid_attn_decode -- the same attention for one new token of each of B sequences, reading
+ * the mixed-precision caches ([ledger]).
+ *   q        [B, H, c] bf16
+ *   comp     compressed cache rows of all sequences; sequence b's entry s is row comp_off[b] + s
+ *   comp_off [B] int64;  pos [B] int64 position t of the new token (N_vis = floor((t+1)/m))
+ *   win      window cache rows, sequence b's rows are b*W .. b*W + win_len[b] - 1, in any order
+ *   win_len  [B] int32 in [0, W]
+ *   idx      [B, k] int32 compressed-entry indices (CSA, -1 = empty) or NULL (HCA: all
+ *            s < min(N_vis, max_nvis))
+ *   o        [B, H, c] bf16;  lse [B, H] fp32 or NULL
+ *   ws       workspace of hybrid_attn_decode_workspace_size(...) bytes (split-K partials)
+ * Limits: c a multiple of 32 and <= 512, H <= 128, W <= 1024.
+ */
+size_t hybrid_attn_decode_workspace_size(int32_t B, int32_t H, int32_t c, int32_t k, int32_t W,
+                                         int64_t max_nvis, int32_t use_idx);
+int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *comp_off,
+                       const int64_t *pos, const csa_kv_rows *win, const int32_t *win_len,
+                       const int32_t *idx, int32_t k, const float *sink, float scale, int32_t B,
+                       int32_t H, int32_t c, int32_t m, int32_t W, int64_t max_nvis, void *o,
+                       float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* ----------------------------------------------------------------------------------------- */
+
+/* Synchronise `stream`, return the device error word (CSA_DEVERR_* bits) in *out and clear it. */
+int csa_device_error(void *stream, int32_t *out);
+
+/* Static description of a status code. */
+const char *csa_status_string(int32_t status);
+
+/* ABI version (major*100 + minor). */
+int32_t csa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,337 @@
+"""GPU parity of every step of the hot path against the fp64 oracle, through the C ABI.
+
+Inputs come from the seeded generators (csa_workloads), never from the CUDA path.  Sizes span
+several tiles and a ragged tail; full-size workloads are in test_gpu_full.py.
+Tolerances: fp32 outputs 2e-5 absolute on O(1) values; bf16 attention outputs 2e-2 max relative
+error per (token, head) row (fp32 accumulation of bf16 / fp8 inputs); storage-format codes
+bit-exact on identical fp32 inputs; top-k sets exact except within 1e-4 relative of the k-th
+score.
+"""
+import numpy as np
+import pytest
+import torch
+
+import csa_workloads as WL
+import oracle as O
+from _util import check_topk, dev, host, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def C(gpu):
+    import compressed_sparse_kv_csa_b200 as C
+    return C
+
+
+def _wl(name, **kw):
+    import dataclasses
+    return dataclasses.replace(WL.WORKLOADS[name], **kw)
+
+
+# ---------------------------------------------------------------------------------------------
+# compression
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,c,dtype", [(1030, 128, "f32"), (4099, 512, "bf16"), (3, 128, "f32"), (4, 32, "bf16")])
+def test_csa_compress(C, T, c, dtype):
+    w = _wl("tiny_csa_fp32", T=T, c=c, dtype=dtype)
+    Ca, Cb, Za, Zb = (WL.draw(w, n, 0, T) for n in ("Ca", "Cb", "Za", "Zb"))
+    B = WL.normal_rows(w.seed, "B/L0/S0", c, 0, 8, std=0.1)
+    ref = O.csa_compress(Ca, Cb, Za, Zb, B, 4)
+    out = torch.empty((T // 4, c), dtype=torch.float32, device="cuda")
+    C.csa_compress(*(dev(x, dtype) for x in (Ca, Cb, Za, Zb)), dev(B), 4, out=out)
+    np.testing.assert_allclose(host(out), ref, atol=2e-5, rtol=0)
+    if T // 4:
+        outb = torch.empty((T // 4, c), dtype=torch.bfloat16, device="cuda")
+        C.csa_compress(*(dev(x, dtype) for x in (Ca, Cb, Za, Zb)), dev(B), 4, out=outb)
+        np.testing.assert_allclose(host(outb), ref, rtol=2 ** -8, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,m", [(1000, 128), (256, 128), (64, 1), (515, 16)])
+def test_hca_compress(C, T, m):
+    w = _wl("hca_prefill_32k", T=T, c=512)
+    Cc, Z = WL.draw(w, "C", 0, T), WL.draw(w, "Z", 0, T)
+    B = WL.normal_rows(w.seed, "B/L0/S0", 512, 0, m, std=0.1)
+    ref = O.hca_compress(Cc, Z, B, m)
+    out = torch.empty((T // m, 512), dtype=torch.float32, device="cuda")
+    C.hca_compress(dev(Cc, "bf16"), dev(Z, "bf16"), dev(B), m, out=out)
+    np.testing.assert_allclose(host(out), ref, atol=2e-5, rtol=0)
+
+
+# ---------------------------------------------------------------------------------------------
+# storage formats
+# ---------------------------------------------------------------------------------------------
+
+def _special_rows(n, c, seed):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((n, c)).astype(np.float32) * np.float32(3)
+    x[0] = 0.0                                   # all-zero row: scale 1 / exponent -127
+    x[1] *= np.float32(1e-30)                    # tiny values
+    x[2] *= np.float32(1e20)                     # large values
+    x[3, ::7] = 448.0                            # exact maximum
+    x[4] = np.float32(6.0) * (2.0 ** g.integers(-3, 3, size=c)).astype(np.float32)  # grid points
+    x[5, :] = np.float32(0.25)                   # ties
+    x[6] = (g.integers(0, 17, size=c) * 0.25).astype(np.float32) * np.sign(g.standard_normal(c)).astype(np.float32)
+    return x
+
+
+def test_quantize_kv_bit_exact(C):
+    x = _special_rows(2053, 512, 7)
+    fp8, rb, sc = O.quant_kv(x, rope=64)
+    kv = C.KvRows.empty(2053, 512, 64, "cuda")
+    C.csa_quantize_kv(dev(x), kv)
+    np.testing.assert_array_equal(kv.fp8.cpu().numpy(), fp8)
+    np.testing.assert_array_equal(kv.rope.view(torch.int16).cpu().numpy().view(np.uint16), rb)
+    np.testing.assert_array_equal(kv.scale.cpu().numpy().view(np.uint32), sc.view(np.uint32))
+
+
+@pytest.mark.parametrize("d", [128, 32])
+def test_quantize_fp4_bit_exact(C, d):
+    x = _special_rows(1031, d, 11)
+    codes, scales = O.quant_fp4(x)
+    f4 = C.Fp4Rows.empty(1031, d, "cuda")
+    C.csa_quantize_fp4(dev(x), f4)
+    np.testing.assert_array_equal(f4.scales.cpu().numpy(), scales)
+    np.testing.assert_array_equal(f4.codes.cpu().numpy(), codes)
+    # bf16 input path
+    xb = WL.on_grid(x, "bf16")
+    codes, scales = O.quant_fp4(xb)
+    C.csa_quantize_fp4(dev(xb, "bf16"), f4)
+    np.testing.assert_array_equal(f4.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(f4.scales.cpu().numpy(), scales)
+
+
+def test_compress_quantise_on_write(C):
+    """Fused cache writes equal the standalone quantisers applied to the same fp32 values, and
+    dequantise to the oracle's compression within the formats' rounding."""
+    T, c = 2048, 512
+    w = _wl("csa_prefill_64k", T=T)
+    Ca, Cb, Za, Zb = (WL.draw(w, n, 0, T) for n in ("Ca", "Cb", "Za", "Zb"))
+    B = WL.normal_rows(w.seed, "B/L0/S0", c, 0, 8, std=0.1)
+    n = T // 4
+    out = torch.empty((n, c), dtype=torch.float32, device="cuda")
+    kv = C.KvRows.empty(n, c, 64, "cuda")
+    C.csa_compress(*(dev(x, "bf16") for x in (Ca, Cb, Za, Zb)), dev(B), 4, out=out, out_kv=kv)
+    kv2 = C.KvRows.empty(n, c, 64, "cuda")
+    C.csa_quantize_kv(out, kv2)
+    assert torch.equal(kv.fp8, kv2.fp8) and torch.equal(kv.scale, kv2.scale)
+    assert torch.equal(kv.rope.view(torch.int16), kv2.rope.view(torch.int16))
+    ref = O.csa_compress(Ca, Cb, Za, Zb, B, 4)
+    deq = O.dequant_kv(kv.fp8.cpu().numpy(), kv.rope.view(torch.int16).cpu().numpy().view(np.uint16),
+                       kv.scale.cpu().numpy())
+    err = np.abs(deq - ref)
+    assert np.all(err[:, :448] <= np.abs(ref[:, :448]) * 2 ** -4 + kv.scale.cpu().numpy()[:, None] * 2 ** -9)
+    assert np.all(err[:, 448:] <= np.abs(ref[:, 448:]) * 2 ** -8 + 1e-6)
+    # FP4 index keys (c = 128)
+    CI = [WL.draw(w, nme, 0, T) for nme in ("CIa", "CIb", "ZIa", "ZIb")]
+    BI = WL.normal_rows(w.seed, "BI/L0/S0", 128, 0, 8, std=0.1)
+    outk = torch.empty((n, 128), dtype=torch.float32, device="cuda")
+    f4 = C.Fp4Rows.empty(n, 128, "cuda")
+    C.csa_compress(*(dev(x, "bf16") for x in CI), dev(BI), 4, out=outk, out_fp4=f4)
+    f4b = C.Fp4Rows.empty(n, 128, "cuda")
+    C.csa_quantize_fp4(outk, f4b)
+    assert torch.equal(f4.codes, f4b.codes) and torch.equal(f4.scales, f4b.scales)
+    refk = O.csa_compress(*CI, BI, 4)
+    deqk = O.dequant_fp4(f4.codes.cpu().numpy(), f4.scales.cpu().numpy())
+    sc = np.repeat(2.0 ** (f4.scales.cpu().numpy().astype(np.float64) - 127), 32, axis=1)
+    assert np.all(np.abs(deqk - refk) <= sc * 1.0 + 1e-6)
+
+
+# ---------------------------------------------------------------------------------------------
+# indexer + top-k
+# ---------------------------------------------------------------------------------------------
+
+def test_indexer_topk_tiny_fp32(C):
+    """The tiny fp32 CSA workload: 1024 queries, 4 index heads of dim 32, 256 keys, k = 64."""
+    w = WL.WORKLOADS["tiny_csa_fp32"]
+    T, H, d, k = w.T, w.H_I, w.d_I, w.k
+    q = WL.draw(w, "qI", 0, T).reshape(T, H, d)
+    K = WL.draw(w, "KI", 0, T // 4)
+    wt = WL.draw(w, "w", 0, T)
+    idx_o, S = O.indexer_topk(q, wt, K, np.arange(T), 4, k)
+    idx = C.indexer_topk(dev(q), dev(wt), dev(K), 4, k, max_nvis=T // 4)
+    nv = O.n_vis(np.arange(T), 4)
+    same = check_topk(idx.cpu().numpy(), idx_o, S, nv, k)
+    assert same >= T - 8
+
+
+def test_indexer_topk_bf16_multi_tile(C):
+    w = WL.WORKLOADS["csa_prefill_64k"]
+    T, H, d, k, m = 1500, 64, 128, 96, 4
+    rows = np.arange(T)
+    q = WL.qI_lowrank(w, 0, T).reshape(T, H, d)
+    K = WL.draw(w, "KI", 0, T // m)
+    wt = WL.draw(w, "w", 0, T)
+    idx_o, S = O.indexer_topk(q, wt, K, rows, m, k)
+    idx = C.indexer_topk(dev(q, "bf16"), dev(wt), dev(K, "bf16"), m, k, max_nvis=T // m)
+    assert check_topk(idx.cpu().numpy(), idx_o, S, O.n_vis(rows, m), k) >= T - 8
+
+
+def test_indexer_topk_fp4_decode_batches(C):
+    """FP4 queries and keys with per-sequence key offsets and positions (decode layout)."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, H, d, k, m = 3, 64, 128, 1024, 4
+    pos = np.array([4 * 3000 + 2, 40001, 4 * 1500 - 1], np.int64)
+    nv = O.n_vis(pos, m)
+    off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+    keys = np.concatenate([WL.draw(w, "KI", 0, int(n), seq=b) for b, n in enumerate(nv)])
+    qx = np.stack([WL.draw(w, "qI", 0, 1, seq=b).reshape(H, d) for b in range(Bn)])
+    wt = np.concatenate([WL.draw(w, "w", 0, 1, seq=b) for b in range(Bn)])
+    kc, ks = O.quant_fp4(keys)
+    qc, qs = O.quant_fp4(qx.reshape(Bn * H, d))
+    Kd = O.dequant_fp4(kc, ks)
+    Qd = O.dequant_fp4(qc, qs).reshape(Bn, H, d)
+    idx_o, S = O.indexer_topk(Qd, wt, Kd, pos, m, k, kbase=off)
+    k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
+    q4 = C.Fp4Rows.empty(Bn * H, d, "cuda")
+    C.csa_quantize_fp4(dev(keys), k4)
+    C.csa_quantize_fp4(dev(qx.reshape(Bn * H, d)), q4)
+    idx = C.indexer_topk(q4, dev(wt), k4, m, k, max_nvis=int(nv.max()),
+                         q_pos=torch.from_numpy(pos).cuda(), key_off=torch.from_numpy(off).cuda())
+    assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
+
+
+def test_topk_ties_short_lists_and_scores(C):
+    T, H, d, k = 300, 2, 32, 50
+    q = np.zeros((T, H, d), np.float32)
+    K = np.random.default_rng(3).standard_normal((100, d)).astype(np.float32)
+    wt = np.ones((T, H), np.float32)
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    idx = C.indexer_topk(dev(q), dev(wt), dev(K), 3, k, max_nvis=100, score_out=sc).cpu().numpy()
+    for t in range(T):
+        nv = min((t + 1) // 3, 100)
+        ke = min(k, nv)
+        assert list(idx[t]) == list(range(ke)) + [-1] * (k - ke)
+    scn = sc.cpu().numpy()
+    assert np.all(scn[idx >= 0] == 0.0) and np.all(np.isneginf(scn[idx < 0]))
+
+
+# ---------------------------------------------------------------------------------------------
+# prefill attention
+# ---------------------------------------------------------------------------------------------
+
+def _prefill_inputs(w, T, n_comp):
+    q = WL.draw(w, "q", 0, T).reshape(T, w.H, w.c)
+    X = WL.draw(w, "X", 0, T)
+    KVc = WL.draw(w, "KV", 0, n_comp)
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    return q, X, KVc, sink
+
+
+def test_prefill_attention_tiny_fp32(C):
+    w = WL.WORKLOADS["tiny_csa_fp32"]
+    T, n_comp = w.T, w.T // 4
+    q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
+    idx = WL.random_topk_idx(w.seed, T, 4, w.k, n_comp)
+    o_ref, lse_ref = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, 4, w.W, idx=idx)
+    lse = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_prefill(dev(q), dev(X), dev(KVc), dev(sink), 1.0, 4, w.W, idx=dev_i(idx), lse=lse)
+    assert row_rel_err(host(o), o_ref).max() < 1e-4
+    np.testing.assert_allclose(host(lse), lse_ref, atol=1e-4)
+
+
+def dev_i(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+@pytest.mark.parametrize("T,W,m", [(1100, 128, 128), (300, 512, 16), (77, 1, 4)])
+def test_prefill_attention_hca_bf16(C, T, W, m):
+    w = _wl("hca_prefill_32k", T=T, W=W, m=m)
+    n_comp = T // m
+    q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
+    o_ref, lse_ref = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, W)
+    lse = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, W, lse=lse)
+    err = row_rel_err(host(o), o_ref)
+    assert err.max() < 2e-2, err.max()
+    np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
+
+
+def test_prefill_attention_csa_bf16_with_invalid_indices(C):
+    w = _wl("csa_prefill_64k", T=700)
+    T, m, k = 700, 4, 64
+    n_comp = T // m
+    q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
+    idx = WL.random_topk_idx(w.seed, T, m, k, n_comp)
+    o_ref, _ = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, w.W, idx=idx)
+    o = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, w.W, idx=dev_i(idx))
+    assert row_rel_err(host(o), o_ref).max() < 2e-2
+    assert C.csa_device_error() == 0
+    bad = idx.copy()
+    bad[5, 0] = n_comp + 3   # out of range: skipped and reported, never read
+    idx2 = bad.copy()
+    idx2[5, 0] = -1
+    o_ref2, _ = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, w.W, idx=idx2, rows=[5])
+    o2 = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, w.W, idx=dev_i(bad))
+    assert C.csa_device_error() & C.CSA_DEVERR_INDEX
+    assert row_rel_err(host(o2)[5], o_ref2[0]).max() < 2e-2
+
+
+# ---------------------------------------------------------------------------------------------
+# decode attention over the mixed caches
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("use_idx", [True, False])
+def test_decode_attention_mixed_cache(C, use_idx):
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, H, c, W, m, k = 5, 64, 512, 128, (4 if use_idx else 128), 256
+    pos = np.array([4 * 900 + 1, 7000, 129, 3, 4 * 2000 - 1], np.int64)
+    nv = O.n_vis(pos, m)
+    off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+    comp = np.concatenate([WL.draw(w, "KV", 0, int(n), seq=b) for b, n in enumerate(nv)])
+    win_len = np.array([128, 77, 0, 4, 128], np.int32)
+    win = np.concatenate([WL.draw(w, "WIN", 0, W, seq=b) for b in range(Bn)])
+    q = np.stack([WL.draw(w, "q", 0, 1, seq=b).reshape(H, c) for b in range(Bn)])
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    idx = None
+    if use_idx:
+        idx = np.full((Bn, k), -1, np.int32)
+        for b in range(Bn):
+            idx[b] = WL.random_topk_idx(w.seed + b, int(pos[b]) + 1, m, k, int(nv[b]), rows=[int(pos[b])])[0]
+    cf, cr, cs = O.quant_kv(comp)
+    wf, wr, ws = O.quant_kv(win)
+    o_ref, lse_ref = O.hybrid_attn_decode(WL.on_grid(q, "bf16"), O.dequant_kv(cf, cr, cs), off, pos,
+                                          O.dequant_kv(wf, wr, ws), win_len, sink, 1.0, m, W, idx=idx)
+    ckv = C.KvRows.empty(len(comp), c, 64, "cuda")
+    wkv = C.KvRows.empty(Bn * W, c, 64, "cuda")
+    C.csa_quantize_kv(dev(comp), ckv)
+    C.csa_quantize_kv(dev(win), wkv)
+    lse = torch.empty((Bn, H), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_decode(dev(WL.on_grid(q, "bf16"), "bf16"), ckv, torch.from_numpy(off).cuda(),
+                             torch.from_numpy(pos).cuda(), wkv, dev_i(win_len), dev(sink), 1.0, m, W,
+                             max_nvis=int(nv.max()), idx=None if idx is None else dev_i(idx), lse=lse)
+    assert row_rel_err(host(o), o_ref).max() < 2e-2
+    np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
+
+
+# ---------------------------------------------------------------------------------------------
+# the tiny CSA layer end to end (compress -> indexer -> top-k -> attention)
+# ---------------------------------------------------------------------------------------------
+
+def test_tiny_csa_layer_end_to_end(C):
+    w = WL.WORKLOADS["tiny_csa_fp32"]
+    T, c, m, H, Hi, di, k, W = w.T, w.c, w.m, w.H, w.H_I, w.d_I, w.k, w.W
+    Ca, Cb, Za, Zb = (WL.draw(w, n, 0, T) for n in ("Ca", "Cb", "Za", "Zb"))
+    B = WL.normal_rows(w.seed, "B/L0/S0", c, 0, 8, std=0.1)
+    qI = WL.draw(w, "qI", 0, T).reshape(T, Hi, di)
+    KI = WL.draw(w, "KI", 0, T // m)
+    wt = WL.draw(w, "w", 0, T)
+    q = WL.draw(w, "q", 0, T).reshape(T, H, c)
+    X = WL.draw(w, "X", 0, T)
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    # oracle
+    KVc = O.csa_compress(Ca, Cb, Za, Zb, B, m)
+    idx_o, S = O.indexer_topk(qI, wt, KI, np.arange(T), m, k)
+    o_ref, _ = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, W, idx=idx_o)
+    # GPU
+    kvc = torch.empty((T // m, c), dtype=torch.float32, device="cuda")
+    C.csa_compress(*(dev(x) for x in (Ca, Cb, Za, Zb)), dev(B), m, out=kvc)
+    idx = C.indexer_topk(dev(qI), dev(wt), dev(KI), m, k, max_nvis=T // m)
+    o = C.hybrid_attn_prefill(dev(q), dev(X), kvc, dev(sink), 1.0, m, W, idx=idx)
+    ig = idx.cpu().numpy()
+    check_topk(ig, idx_o, S, O.n_vis(np.arange(T), m), k)
+    same = np.array([set(ig[t].tolist()) == set(idx_o[t].tolist()) for t in range(T)])
+    assert same.sum() >= T - 8
+    err = row_rel_err(host(o)[same], o_ref[same])
+    assert err.max() < 1e-4, err.max()
