@@ -197,28 +197,48 @@ WORKLOADS = {"hca_prefill_32k": HcaPrefill}
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_hca_sample(w, n_tokens: int, seed_rank: int = 0):
-    """Time the oracle on a bounded sample of the HCA layer: the full compression (amortised
-    over T) plus attention of n_tokens query tokens spread over the sequence.
-    Returns (tokens/s, seconds, description)."""
-    import oracle as O
-    T, c, H, m, W = w.T, w.c, w.H, w.m, w.W
-    Cc = WL.draw(w, "C", 0, T, seq=seed_rank)
-    Z = WL.draw(w, "Z", 0, T, seq=seed_rank)
-    B = WL.normal_rows(w.seed, f"B/L0/S{seed_rank}", c, 0, m, std=w.bias_std)
-    rows = np.linspace(0, T - 1, n_tokens).astype(np.int64)
-    qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1, seq=seed_rank)[0] for t in rows]).reshape(n_tokens, H, c)
-    X = WL.draw(w, "X", 0, T, seq=seed_rank)
-    sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
-    t0 = time.perf_counter()
-    KV = O.hca_compress(Cc, Z, B, m)
-    t1 = time.perf_counter()
-    O.hybrid_attn_prefill(qs, X, KV, sink, 1.0, m, W, rows=rows)
-    t2 = time.perf_counter()
-    per_token = (t1 - t0) / T + (t2 - t1) / n_tokens
-    desc = (f"full hca_compress of T={T} (amortised per token) + hybrid attention of {n_tokens} query tokens "
-            f"evenly spaced over the layer")
-    return 1.0 / per_token, (t2 - t0), desc
+class OracleHca:
+    """The oracle on a bounded sample of the HCA layer: the full compression (amortised over T)
+    plus attention of n_tokens query tokens evenly spaced over the sequence.  Inputs are drawn
+    once (untimed); run() times the oracle's own work."""
+
+    def __init__(self, w, n_tokens: int, seed_rank: int = 0):
+        T, c, H, m = w.T, w.c, w.H, w.m
+        self.w, self.n = w, n_tokens
+        self.Cc = WL.draw(w, "C", 0, T, seq=seed_rank)
+        self.Z = WL.draw(w, "Z", 0, T, seq=seed_rank)
+        self.B = WL.normal_rows(w.seed, f"B/L0/S{seed_rank}", c, 0, m, std=w.bias_std)
+        self.rows = np.linspace(0, T - 1, n_tokens).astype(np.int64)
+        self.qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1, seq=seed_rank)[0]
+                            for t in self.rows]).reshape(n_tokens, H, c)
+        self.X = WL.draw(w, "X", 0, T, seq=seed_rank)
+        self.sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
+
+    def run(self):
+        """Returns (tokens/s, seconds of oracle work, compress seconds, attention seconds)."""
+        import oracle as O
+        w = self.w
+        t0 = time.perf_counter()
+        KV = O.hca_compress(self.Cc, self.Z, self.B, w.m)
+        t1 = time.perf_counter()
+        O.hybrid_attn_prefill(self.qs, self.X, KV, self.sink, 1.0, w.m, w.W, rows=self.rows)
+        t2 = time.perf_counter()
+        per_token = (t1 - t0) / w.T + (t2 - t1) / self.n
+        return 1.0 / per_token, t2 - t0, t1 - t0, t2 - t1
+
+    def describe(self):
+        return (f"full hca_compress of T={self.w.T} (amortised per token) + hybrid attention of {self.n} "
+                f"query tokens evenly spaced over the layer")
+
+
+def oracle_hca_sample(w, target_s: float = 10.0):
+    """cpu_baseline leg: calibrate the sample so the oracle's attention work takes ~target_s."""
+    probe = OracleHca(w, 16)
+    _, _, _, t_attn = probe.run()
+    n = int(min(4096, max(16, target_s / max(t_attn / 16, 1e-6))))
+    job = OracleHca(w, n)
+    tps, secs, _, _ = job.run()
+    return tps, secs, job.describe()
 
 
 # ---------------------------------------------------------------------------------------------
@@ -329,9 +349,7 @@ def main():
         }
         if not args.no_cpu_baseline and world == 1:
             import oracle as O
-            tps, secs, desc = oracle_hca_sample(w, 16)
-            n = int(min(4096, max(16, 12.0 / max(secs, 1e-3) * 16)))
-            tps, secs, desc = oracle_hca_sample(w, n)
+            tps, secs, desc = oracle_hca_sample(w)
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
                                     "sample": desc, "seconds": secs}
         print(json.dumps(line), flush=True)
@@ -345,12 +363,13 @@ def reference_arm(args, w, world, rank):
     if rank != 0:
         return
     import oracle as O
-    n = 64
+    job = OracleHca(w, 256)
+    desc = job.describe()
     for _ in range(max(args.warmup, 3)):
-        oracle_hca_sample(w, n)
+        job.run()
     vals, secs = [], []
     for _ in range(args.steps):
-        tps, s, desc = oracle_hca_sample(w, n)
+        tps, s, _, _ = job.run()
         vals.append(tps)
         secs.append(s)
     value = statistics.median(vals)

@@ -96,6 +96,7 @@ int csa_compress(const void *Ca, const void *Cb, const void *Za, const void *Zb,
     if (!Ca || !Cb || !Za || !Zb || !B || T < 0 || m < 1 || m > 64 || !dtype_ok(in_dtype))
         return CSA_ERR_INVALID_ARG;
     if (c <= 0 || c % 4 || c > 2048) return CSA_ERR_UNSUPPORTED;
+    if (T / m == 0) return CSA_OK; // no complete block: nothing to write
     if (!out && !out_kv && !out_fp4) return CSA_ERR_INVALID_ARG;
     if (out && !dtype_ok(out_dtype)) return CSA_ERR_INVALID_ARG;
     if (!aligned16(B) || !aligned16(Ca) || !aligned16(Cb) || !aligned16(Za) || !aligned16(Zb))
@@ -118,6 +119,7 @@ int hca_compress(const void *C, const void *Z, const float *B, int64_t T, int32_
 {
     if (!C || !Z || !B || T < 0 || m < 1 || m > 1024 || !dtype_ok(in_dtype)) return CSA_ERR_INVALID_ARG;
     if (c <= 0 || c % 4 || c > 2048) return CSA_ERR_UNSUPPORTED;
+    if (T / m == 0) return CSA_OK; // no complete block: nothing to write
     if (!out && !out_kv) return CSA_ERR_INVALID_ARG;
     if (out && !dtype_ok(out_dtype)) return CSA_ERR_INVALID_ARG;
     if (!aligned16(B) || !aligned16(C) || !aligned16(Z) || (out && !aligned16(out))) return CSA_ERR_INVALID_ARG;

@@ -99,7 +99,7 @@ typedef struct csa_fp4_rows {
  *   Ca, Cb, Za, Zb  [T, c] in `in_dtype` (CSA_F32 or CSA_BF16)
  *   B               [2m, c] fp32: rows 0..m-1 = B^a (current block), rows m..2m-1 = B^b
  *   T >= 0, 1 <= m <= 64, c a multiple of 4 and <= 2048
- * Outputs (any subset, at least one non-NULL):
+ * Outputs (any subset; at least one non-NULL unless floor(T/m) == 0, which writes nothing):
  *   out      [floor(T/m), c] in `out_dtype` (CSA_F32 or CSA_BF16)
  *   out_kv   mixed FP8/BF16 rows (quantise-on-write), out_kv->n >= floor(T/m), ->c == c
  *   out_fp4  FP4 rows (quantise-on-write, for index keys), ->n >= floor(T/m), ->d == c
