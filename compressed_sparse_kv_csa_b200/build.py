@@ -1,6 +1,6 @@
 """Build libcsa.so (all CUDA sources under csrc/) for sm_100a with nvcc, in-tree.
 
-    python -m compressed_sparse_kv_csa_b200.build [--force]
+    python compressed_sparse_kv_csa_b200/build.py [--force]   (by path: importing the package loads the .so)
 
 Objects are compiled in parallel into _build/ and linked into
 compressed_sparse_kv_csa_b200/libcsa.so.  A source, header or flag change triggers a rebuild.

@@ -12,8 +12,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def C():
-    from compressed_sparse_kv_csa_b200 import build
-    build.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "csa_build", os.path.join(ROOT, "compressed_sparse_kv_csa_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
     import compressed_sparse_kv_csa_b200 as C
     return C
 
