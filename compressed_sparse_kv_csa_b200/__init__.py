@@ -53,7 +53,7 @@ class _Fp4Rows(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libcsa.so not found at {LIB_PATH}: build it with "
-                          "`python -m compressed_sparse_kv_csa_b200.build` (nvcc, sm_100a)")
+                          "`python compressed_sparse_kv_csa_b200/build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     P_kv, P_f4 = ctypes.POINTER(_KvRows), ctypes.POINTER(_Fp4Rows)
@@ -70,6 +70,9 @@ def _load():
         "hybrid_attn_decode_workspace_size": ([i32, i32, i32, i32, i32, i64, i32], sz),
         "hybrid_attn_decode": ([vp, P_kv, vp, vp, P_kv, vp, vp, i32, vp, f32, i32, i32, i32, i32, i32, i64,
                                 vp, vp, vp, sz, vp], ctypes.c_int),
+        "indexer_topk_static_capacity": ([], sz),
+        "indexer_topk_static": ([vp, vp, vp, i32, vp, vp, i64, i64, i32, i32, i32, i32, i64, vp, vp, vp],
+                                ctypes.c_int),
         "csa_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
         "csa_status_string": ([i32], ctypes.c_char_p),
         "csa_abi_version": ([], i32),
@@ -245,6 +248,31 @@ def indexer_topk(q, w, keys, m: int, k: int, max_nvis: int, q_pos=None, key_off=
                            max_nvis, _ptr(idx_out), _ptr(score_out), _ptr(workspace), workspace.numel(),
                            _stream(stream))
     _check("indexer_topk", st)
+    return idx_out
+
+
+CSA_ERR_SCRATCH_CAPACITY = -6
+
+
+def indexer_topk_static(q, w, keys, m: int, k: int, max_nvis: int, q_pos=None, key_off=None, n_keys=None,
+                        idx_out=None, score_out=None, stream=None):
+    """indexer_topk without a workspace, for callers that cannot allocate device memory: the
+    score scratch is the library's static device array (see include/csa.h for its capacity,
+    first-call set-up and why overlapping calls must be serialised)."""
+    if isinstance(q, Fp4Rows):
+        fmt, Nq, H_I, d_I = CSA_FP4, w.shape[0], w.shape[1], q.d
+        n_keys = keys.n if n_keys is None else n_keys
+        qarg, karg, device = ctypes.byref(q._c()), ctypes.byref(keys._c()), q.codes.device
+    else:
+        fmt = _dtype_code(q)
+        Nq, H_I, d_I = q.shape
+        n_keys = keys.shape[0] if n_keys is None else n_keys
+        qarg, karg, device = _ptr(q), _ptr(keys), q.device
+    if idx_out is None:
+        idx_out = torch.empty((Nq, k), dtype=torch.int32, device=device)
+    st = _lib.indexer_topk_static(qarg, _ptr(w), karg, fmt, _ptr(q_pos), _ptr(key_off), n_keys, Nq, H_I, d_I,
+                                  m, k, max_nvis, _ptr(idx_out), _ptr(score_out), _stream(stream))
+    _check("indexer_topk_static", st)
     return idx_out
 
 

@@ -69,6 +69,7 @@ const char *csa_status_string(int32_t s)
     case CSA_ERR_UNSUPPORTED: return "unsupported shape or type";
     case CSA_ERR_CUDA: return "CUDA launch error";
     case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA_ERR_SCRATCH_CAPACITY: return "request exceeds the static scratch capacity";
     default: return "unknown status";
     }
 }

@@ -167,6 +167,29 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
                  int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis,
                  int32_t *idx_out, float *score_out, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * indexer_topk_static -- indexer_topk for callers that cannot allocate device memory (for
+ * example runtimes that reserve the device memory for their own pools up front and give plugins
+ * no allocator).  The pages have no counterpart: this is a library convenience.
+ *
+ * Same arguments, semantics and results as indexer_topk, without the workspace: the score
+ * scratch is a file-scope device array of indexer_topk_static_capacity() = 4,194,304 fp32 scores
+ * (16 MiB), which every GPU that loads this library holds until the process exits.  Requests
+ * with Nq * ceil4(max_nvis) above that capacity return CSA_ERR_SCRATCH_CAPACITY before anything
+ * is launched.  No cudaMalloc, cudaFree or allocating library routine is called.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture begins.
+ *   - All calls on a device share the one array, which keeps the last call's contents.  Nothing
+ *     in it needs to start at zero (each call writes every score it reads), but calls whose
+ *     kernels overlap on the GPU (different streams without ordering) race on it: serialise them.
+ */
+#define CSA_ERR_SCRATCH_CAPACITY (-6) /* request exceeds the static scratch of *_static calls */
+size_t indexer_topk_static_capacity(void);
+int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t fmt,
+                        const int64_t *q_pos, const int64_t *key_off, int64_t n_keys, int64_t Nq,
+                        int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis,
+                        int32_t *idx_out, float *score_out, void *stream);
+
 /* ----------------------------------------------------------------------------------------- */
 
 /*
