@@ -252,8 +252,12 @@ def main():
     ap.add_argument("--workload", default="hca_prefill_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None, help="override the token count (profiling a smaller case)")
     args = ap.parse_args()
     w = WL.WORKLOADS[args.workload]
+    if args.T is not None:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.T)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

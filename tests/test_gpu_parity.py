@@ -248,6 +248,25 @@ def test_prefill_attention_hca_bf16(C, T, W, m):
     np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
 
 
+@pytest.mark.parametrize("T,m,k", [(1, 4, None), (130, 128, None), (2000, 16, None), (300, 4, 512), (157, 4, 200)])
+def test_prefill_attention_tensor_core_shapes(C, T, m, k):
+    """64 heads x 512 channels, bf16, window 128: the tcgen05 path.  Covers a single token, fewer
+    tokens than SMs, several tokens per CTA, 1-2 compressed tiles, 4 top-k tiles with many empty
+    (-1) slots and a top-k length that is not a multiple of the 128-key tile."""
+    w = _wl("csa_prefill_64k", T=T, m=m)
+    n_comp = max(T // m, 1)
+    q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
+    idx = WL.random_topk_idx(w.seed, T, m, k, n_comp) if k else None
+    o_ref, lse_ref = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, 128, idx=idx)
+    lse = torch.empty((T, 64), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, 128,
+                              idx=None if idx is None else dev_i(idx), lse=lse)
+    err = row_rel_err(host(o), o_ref)
+    assert err.max() < 2e-2, err.max()
+    np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
+    assert C.csa_device_error() == 0
+
+
 def test_prefill_attention_csa_bf16_with_invalid_indices(C):
     w = _wl("csa_prefill_64k", T=700)
     T, m, k = 700, 4, 64
