@@ -190,7 +190,147 @@ class HcaPrefill:
         self.h_out.copy_(self.o, non_blocking=True)
 
 
-WORKLOADS = {"hca_prefill_32k": HcaPrefill}
+class CsaPrefill:
+    """One CSA layer prefill (T = 65536): csa_compress of the KV entries and of the index keys,
+    indexer_topk (64 index heads x 128, k = 512) and hybrid_attn_prefill over window + top-k."""
+
+    def __init__(self, w, rank, torch, C, device):
+        self.w, self.torch, self.C, self.dev = w, torch, C, device
+        T, c, H, m, Hi, di = w.T, w.c, w.H, w.m, w.H_I, w.d_I
+        bf = torch.bfloat16
+        self.kv_in = [torch.empty((T, c), dtype=bf, device=device) for _ in range(4)]
+        self.ki_in = [torch.empty((T, di), dtype=bf, device=device) for _ in range(4)]
+        for name, t in zip(("Ca", "Cb", "Za", "Zb"), self.kv_in):
+            gen_rows_bf16(w, name, T, c, torch, t, seq=rank)
+        for name, t in zip(("CIa", "CIb", "ZIa", "ZIb"), self.ki_in):
+            gen_rows_bf16(w, name, T, di, torch, t, seq=rank)
+        self.X = torch.empty((T, c), dtype=bf, device=device)
+        gen_rows_bf16(w, "X", T, c, torch, self.X, seq=rank)
+        self.q = torch.empty((T, H, c), dtype=bf, device=device)
+        gen_rows_bf16(w, "q", T, H * c, torch, self.q.view(T, H * c), seq=rank, chunk=256)
+        self.qI = torch.empty((T, Hi, di), dtype=bf, device=device)
+        for r0 in range(0, T, 4096):
+            self.qI.view(T, Hi * di)[r0:r0 + 4096].copy_(torch.from_numpy(WL.qI_lowrank(w, r0, min(T, r0 + 4096))).to(bf))
+        self.wI = torch.from_numpy(WL.draw(w, "w", 0, T, seq=rank)).to(device)
+        self.B = torch.from_numpy(WL.normal_rows(w.seed, f"B/L0/S{rank}", c, 0, 2 * m, std=w.bias_std)).to(device)
+        self.BI = torch.from_numpy(WL.normal_rows(w.seed, f"BI/L0/S{rank}", di, 0, 2 * m, std=w.bias_std)).to(device)
+        self.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, seq=rank)[0]).to(device)
+        n = T // m
+        self.kvc = torch.empty((n, c), dtype=bf, device=device)
+        self.keys = torch.empty((n, di), dtype=bf, device=device)
+        self.idx = torch.empty((T, w.k), dtype=torch.int32, device=device)
+        self.ws = torch.empty((C.indexer_topk_workspace_size(T, n, w.k),), dtype=torch.uint8, device=device)
+        self.o = torch.empty_like(self.q)
+        t = np.arange(T, dtype=np.int64)
+        self.flops = float(np.minimum((t + 1) // m, n).sum()) * Hi * di * 2.0  # indexer (dominant)
+        self.flops_attn = attn_flops(T, H, c, w.W, m, n, w.k)
+        self.tokens = T
+        self.launches_per_step = 5  # compress x2, indexer scores, top-k, attention
+        self.kernel_name = "indexer_topk (scores)"
+
+    def step(self, ev=None):
+        C, w = self.C, self.w
+        C.csa_compress(*self.kv_in, self.B, w.m, out=self.kvc)
+        C.csa_compress(*self.ki_in, self.BI, w.m, out=self.keys)
+        if ev is not None:
+            ev[0].record()
+        C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=w.T // w.m, idx_out=self.idx,
+                       workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+        C.hybrid_attn_prefill(self.q, self.X, self.kvc, self.sink, 1.0, w.m, w.W, idx=self.idx, o=self.o)
+
+    def setup_e2e(self):
+        torch = self.torch
+        self.dev_in = self.kv_in + self.ki_in + [self.X, self.q, self.qI, self.wI]
+        self.h_in = [t.cpu().pin_memory() for t in self.dev_in]
+        self.h_out = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = self.o.numel() * self.o.element_size()
+
+    def step_e2e(self):
+        for d, h in zip(self.dev_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.o, non_blocking=True)
+
+
+class CsaDecode1M:
+    """CSA decode at 1M context: 8 sequences, one new token each at t = 1,048,576 against
+    262,144 compressed entries (FP8 + BF16 KV rows, FP4 index keys), k = 1024, window 128.
+    One step = indexer_topk (FP4 key scan + top-k) + hybrid_attn_decode."""
+
+    def __init__(self, w, rank, torch, C, device):
+        self.w, self.torch, self.C, self.dev = w, torch, C, device
+        Bn, H, c, Hi, di, W, m = w.B, w.H, w.c, w.H_I, w.d_I, w.W, w.m
+        t = w.T
+        nv = (t + 1) // m
+        self.nv = nv
+        self.comp = C.KvRows.empty(Bn * nv, c, w.rope, device)
+        self.keys = C.Fp4Rows.empty(Bn * nv, di, device)
+        chunk = 16384
+        for b in range(Bn):
+            for r0 in range(0, nv, chunk):
+                r1 = min(nv, r0 + chunk)
+                x = torch.from_numpy(WL.draw(w, "KV", r0, r1, seq=b + 8 * rank)).to(device)
+                C.csa_quantize_kv(x, C.KvRows(self.comp.fp8[b * nv + r0:b * nv + r1], self.comp.rope[b * nv + r0:b * nv + r1],
+                                              self.comp.scale[b * nv + r0:b * nv + r1]))
+                k = torch.from_numpy(WL.draw(w, "KI", r0, r1, seq=b + 8 * rank)).to(device)
+                C.csa_quantize_fp4(k, C.Fp4Rows(self.keys.codes[b * nv + r0:b * nv + r1],
+                                                self.keys.scales[b * nv + r0:b * nv + r1]))
+        win = torch.from_numpy(np.concatenate([WL.draw(w, "WIN", 0, W, seq=b + 8 * rank) for b in range(Bn)])).to(device)
+        self.win = C.KvRows.empty(Bn * W, c, w.rope, device)
+        C.csa_quantize_kv(win, self.win)
+        self.q = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, seq=b + 8 * rank).reshape(H, c)
+                                            for b in range(Bn)])).to(torch.bfloat16).to(device)
+        qx = torch.from_numpy(np.concatenate([WL.draw(w, "qI", 0, 1, seq=b + 8 * rank).reshape(Hi, di)
+                                              for b in range(Bn)])).to(device)
+        self.qI = C.Fp4Rows.empty(Bn * Hi, di, device)
+        C.csa_quantize_fp4(qx, self.qI)
+        self.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, seq=b + 8 * rank) for b in range(Bn)])).to(device)
+        self.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, seq=rank)[0]).to(device)
+        self.pos = torch.full((Bn,), t, dtype=torch.int64, device=device)
+        self.key_off = torch.arange(Bn, dtype=torch.int64, device=device) * nv
+        self.win_len = torch.full((Bn,), W, dtype=torch.int32, device=device)
+        self.idx = torch.empty((Bn, w.k), dtype=torch.int32, device=device)
+        self.ws = torch.empty((C.indexer_topk_workspace_size(Bn, nv, w.k),), dtype=torch.uint8, device=device)
+        self.wsd = torch.empty((C.hybrid_attn_decode_workspace_size(Bn, H, c, w.k, W, nv, True),), dtype=torch.uint8,
+                               device=device)
+        self.o = torch.empty_like(self.q)
+        torch.cuda.synchronize()
+        self.bytes = float(Bn * nv * (di // 2 + di // 32))           # FP4 key scan (dominant)
+        self.bytes_step = self.bytes + Bn * (w.k + W) * (c - w.rope + 2 * w.rope + 4) + 2 * Bn * H * c * 2
+        self.tokens = Bn
+        self.launches_per_step = 4
+        self.kernel_name = "indexer_topk (FP4 scan + top-k)"
+
+    def step(self, ev=None):
+        C, w = self.C, self.w
+        if ev is not None:
+            ev[0].record()
+        C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=self.nv, q_pos=self.pos,
+                       key_off=self.key_off, idx_out=self.idx, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+        C.hybrid_attn_decode(self.q, self.comp, self.key_off, self.pos, self.win, self.win_len, self.sink, 1.0,
+                             w.m, w.W, max_nvis=self.nv, idx=self.idx, o=self.o, workspace=self.wsd)
+
+    def setup_e2e(self):
+        torch = self.torch
+        self.dev_in = [self.q, self.qI.codes, self.qI.scales, self.wI, self.pos]
+        self.h_in = [t.cpu().pin_memory() for t in self.dev_in]
+        self.h_out = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = self.o.numel() * self.o.element_size()
+
+    def step_e2e(self):
+        for d, h in zip(self.dev_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.o, non_blocking=True)
+
+
+WORKLOADS = {"hca_prefill_32k": HcaPrefill, "csa_prefill_64k": CsaPrefill, "csa_decode_1m": CsaDecode1M}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -325,7 +465,27 @@ def main():
 
     if rank == 0:
         pk, src = peaks()
-        achieved = job.flops / (kern_ms * 1e-3) / 1e12
+        if hasattr(job, "bytes"):  # HBM-bound dominant kernel
+            achieved = job.bytes / (kern_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": job.kernel_name, "achieved": achieved, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": f"{src} HBM copy",
+                    "traffic": None, "bytes_per_launch": job.bytes, "launch_ms": kern_ms}
+        else:
+            achieved = job.flops / (kern_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "kernel": getattr(job, "kernel_name", "hybrid_attn_prefill"),
+                    "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / pk["bf16_tflops"], "peak_source": f"{src} dense bf16 burst",
+                    "traffic": None, "flops_per_launch": job.flops, "launch_ms": kern_ms}
+        cfg = {"workload": args.workload, "T": w.T, "c": w.c, "rope_dims": w.rope, "m": w.m, "H": w.H, "W": w.W,
+               "parallelism": f"replicas x{world}"}
+        if w.kind == "csa_decode":
+            cfg.update({"B": w.B, "n_comp_per_seq": (w.T + 1) // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+                        "l2": "FP4 key scan (143 MB) and KV cache (1.2 GB) larger than L2"})
+        elif w.kind == "csa_prefill":
+            cfg.update({"n_comp": w.T // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+                        "l2": "inputs larger than L2 (q alone is 4.3 GB)"})
+        else:
+            cfg.update({"n_comp": w.T // w.m, "l2": f"inputs larger than L2 (q alone is {w.T * w.H * w.c * 2 / 1e9:.1f} GB)"})
         line = {
             "metric": METRIC,
             "value": world * job.tokens / (ms * 1e-3),
@@ -338,20 +498,15 @@ def main():
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) inputs on the bf16 grid, no trained weights)",
-            "config": {"workload": args.workload, "T": w.T, "c": w.c, "rope_dims": w.rope, "m": w.m, "H": w.H,
-                       "W": w.W, "n_comp": w.T // w.m, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (q alone is 2.1 GB)"},
-            "roofline": {"bound": "tensor", "kernel": "hybrid_attn_prefill", "achieved": achieved,
-                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                         "peak_source": f"{src} dense bf16 burst", "traffic": None,
-                         "flops_per_launch": job.flops, "launch_ms": kern_ms},
+            "data": "synthetic (seeded N(0,1) inputs, bf16 grid / FP8 / FP4 caches, no trained weights)",
+            "config": cfg,
+            "roofline": roof,
             "e2e": {"value": world * job.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": job.h2d, "d2h_bytes_per_step": job.d2h, "ms_per_step": e2e_ms},
             "clocks": clk.summary(),
             "gpu_launches": job.launches_per_step * args.steps,
         }
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and args.workload == "hca_prefill_32k":
             import oracle as O
             tps, secs, desc = oracle_hca_sample(w)
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",

@@ -23,6 +23,7 @@ int *dev_error_word()
 }
 cudaError_t launch_attn_prefill_generic(const PrefillArgs &a, cudaStream_t st);
 cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled);
+cudaError_t launch_indexer_scores_tc(const IndexerArgs &a, cudaStream_t st, bool *handled);
 } // namespace csa
 
 using namespace csa;
@@ -200,7 +201,9 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
     a.score_out = score_out;
     a.err = dev_error_word();
     if (Nq == 0) return CSA_OK;
-    cudaError_t e = launch_indexer_scores(a, S(stream));
+    bool handled = false;
+    cudaError_t e = launch_indexer_scores_tc(a, S(stream), &handled);
+    if (!handled) e = launch_indexer_scores(a, S(stream));
     if (e != cudaSuccess) return CSA_ERR_CUDA;
     return status_of(launch_topk(a, S(stream)));
 }

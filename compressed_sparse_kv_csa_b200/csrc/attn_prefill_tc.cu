@@ -29,8 +29,7 @@
 #include "common.cuh"
 #include "tc_common.cuh"
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
+#include "tma_host.cuh"
 
 namespace csa {
 
@@ -421,31 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prefill_tc_kernel(PrefillArg
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// bf16 matrix [rows, 512] with a 1024-byte row stride, boxes of 64 channels x box_rows rows.
 bool encode_rows512(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows)
 {
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kC, rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kC * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tma::encode_bf16_rows(m, base, rows, kC, box_rows);
 }
 
 } // namespace

@@ -208,5 +208,10 @@ def random_topk_idx(seed: int, T: int, m: int, k: int, n_comp: int, rows=None) -
             continue
         g = rng(seed, "topk_idx", int(t))
         n = min(k, nv)
-        out[i, :n] = g.choice(nv, size=n, replace=False)
+        if nv <= 4 * k:
+            out[i, :n] = g.permutation(nv)[:n]
+        else:  # distinct draws by rejection: first n distinct values of a long uniform stream
+            cand = g.integers(0, nv, size=4 * k)
+            _, first = np.unique(cand, return_index=True)
+            out[i, :n] = cand[np.sort(first)][:n]
     return out

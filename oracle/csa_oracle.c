@@ -136,9 +136,10 @@ void orc_hca_compress(const double *C, const double *Z, const double *B, int64_t
 void orc_indexer_scores(const double *q, const double *w, const double *K, const int64_t *kbase,
                         const int64_t *nvis, int64_t Nq, int H, int d, int64_t ldS, double *S)
 {
-#pragma omp parallel for schedule(dynamic, 1)
+    /* every (row, entry) score is independent: parallelise over entries within each row */
     for (int64_t r = 0; r < Nq; r++) {
         const double *qr = q + r * (int64_t)H * d;
+#pragma omp parallel for schedule(static)
         for (int64_t s = 0; s < nvis[r]; s++) {
             const double *ks = K + (kbase[r] + s) * (int64_t)d;
             double acc = 0.0;

@@ -1,0 +1,217 @@
+"""GPU parity at the workloads' full sizes, on outputs the oracle computes row by row.
+
+* hca_prefill_32k  (T = 32768, the workload bench.py times): compression of all 256 entries,
+  attention rows 0..255, 256 seeded random rows and the rows around compressed-block boundaries.
+* csa_prefill_64k  (T = 65536): both compressions in full; indexer top-k on 48 sampled rows
+  (block boundaries, random, last rows); attention on sampled rows with a seeded top-k list.
+* csa_decode_1m    (8 sequences at t = 1,048,576, 262,144 entries each): every sequence's FP4 key
+  scan + top-k, and the attention of rows whose GPU and oracle top-k sets agree.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import csa_workloads as WL
+import oracle as O
+from _util import check_topk, dev, host, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def C(gpu):
+    import compressed_sparse_kv_csa_b200 as C
+    return C
+
+
+def _fill(w, name, rows, ncols, dtype=torch.bfloat16, chunk=2048):
+    out = torch.empty((rows, ncols), dtype=dtype, device="cuda")
+    for r0 in range(0, rows, chunk):
+        r1 = min(rows, r0 + chunk)
+        out[r0:r1].copy_(torch.from_numpy(WL.draw(w, name, r0, r1)).to(dtype))
+    return out
+
+
+def _sample_rows(T, m, seed, n_random=256, head=256):
+    g = np.random.default_rng(seed)
+    rows = set(range(min(head, T)))
+    rows |= set(g.integers(0, T, size=n_random).tolist())
+    for b in (1, 2, T // m // 2, T // m - 1):   # around compressed-block boundaries
+        for d in (-2, -1, 0, 1):
+            t = b * m + d
+            if 0 <= t < T:
+                rows.add(t)
+    rows |= {T - 2, T - 1}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def test_hca_prefill_32k_full(C):
+    w = WL.WORKLOADS["hca_prefill_32k"]
+    T, c, H, m, W = w.T, w.c, w.H, w.m, w.W
+    Cc, Z, X = _fill(w, "C", T, c), _fill(w, "Z", T, c), _fill(w, "X", T, c)
+    q = _fill(w, "q", T, H * c, chunk=256).view(T, H, c)
+    B = WL.normal_rows(w.seed, "B/L0/S0", c, 0, m, std=w.bias_std)
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    kv = torch.empty((T // m, c), dtype=torch.float32, device="cuda")
+    C.hca_compress(Cc, Z, dev(B), m, out=kv)
+    kvb = torch.empty((T // m, c), dtype=torch.bfloat16, device="cuda")
+    C.hca_compress(Cc, Z, dev(B), m, out=kvb)
+    lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_prefill(q, X, kvb, dev(sink), 1.0, m, W, lse=lse)
+    torch.cuda.synchronize()
+    # compression: every entry
+    ref_kv = O.hca_compress(WL.draw(w, "C", 0, T), WL.draw(w, "Z", 0, T), B, m)
+    np.testing.assert_allclose(host(kv), ref_kv, atol=2e-5, rtol=0)
+    # attention: sampled rows, on the bf16 entries the layer stores
+    rows = _sample_rows(T, m, 11)
+    qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1)[0] for t in rows]).reshape(len(rows), H, c)
+    o_ref, lse_ref = O.hybrid_attn_prefill(qs, WL.draw(w, "X", 0, T), host(kvb), sink, 1.0, m, W, rows=rows)
+    og = host(o[torch.from_numpy(rows).cuda()])
+    err = row_rel_err(og, o_ref)
+    assert err.max() < 2e-2, err.max()
+    np.testing.assert_allclose(host(lse)[rows], lse_ref, atol=2e-3)
+    assert C.csa_device_error() == 0
+
+
+@pytest.fixture(scope="module")
+def csa64k():
+    return WL.WORKLOADS["csa_prefill_64k"]
+
+
+def test_csa_prefill_64k_compress_full(C, csa64k):
+    w = csa64k
+    T, c, m = w.T, w.c, w.m
+    ins = [_fill(w, n, T, c) for n in ("Ca", "Cb", "Za", "Zb")]
+    B = WL.normal_rows(w.seed, "B/L0/S0", c, 0, 2 * m, std=w.bias_std)
+    out = torch.empty((T // m, c), dtype=torch.float32, device="cuda")
+    C.csa_compress(*ins, dev(B), m, out=out)
+    ref = O.csa_compress(*(WL.draw(w, n, 0, T) for n in ("Ca", "Cb", "Za", "Zb")), B, m)
+    np.testing.assert_allclose(host(out), ref, atol=2e-5, rtol=0)
+    # index keys (d_I = 128) with FP4 quantise-on-write, checked against the standalone quantiser
+    insI = [_fill(w, n, T, w.d_I) for n in ("CIa", "CIb", "ZIa", "ZIb")]
+    BI = WL.normal_rows(w.seed, "BI/L0/S0", w.d_I, 0, 2 * m, std=w.bias_std)
+    outI = torch.empty((T // m, w.d_I), dtype=torch.float32, device="cuda")
+    f4 = C.Fp4Rows.empty(T // m, w.d_I, "cuda")
+    C.csa_compress(*insI, dev(BI), m, out=outI, out_fp4=f4)
+    refI = O.csa_compress(*(WL.draw(w, n, 0, T) for n in ("CIa", "CIb", "ZIa", "ZIb")), BI, m)
+    np.testing.assert_allclose(host(outI), refI, atol=2e-5, rtol=0)
+    f4b = C.Fp4Rows.empty(T // m, w.d_I, "cuda")
+    C.csa_quantize_fp4(outI, f4b)
+    assert torch.equal(f4.codes, f4b.codes) and torch.equal(f4.scales, f4b.scales)
+
+
+def test_csa_prefill_64k_indexer_sampled(C, csa64k):
+    w = csa64k
+    T, m, k, Hi, di = w.T, w.m, w.k, w.H_I, w.d_I
+    n = T // m
+    K = WL.draw(w, "KI", 0, n)                     # bf16-grid index keys (given directly)
+    qI = torch.empty((T, Hi * di), dtype=torch.bfloat16, device="cuda")
+    for r0 in range(0, T, 4096):
+        qI[r0:r0 + 4096].copy_(torch.from_numpy(WL.qI_lowrank(w, r0, r0 + 4096)).to(torch.bfloat16))
+    wt = WL.draw(w, "w", 0, T)
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    idx = C.indexer_topk(qI.view(T, Hi, di), dev(wt), dev(K, "bf16"), m, k, max_nvis=n, score_out=sc)
+    torch.cuda.synchronize()
+    g = np.random.default_rng(5)
+    rows = np.array(sorted({3, 4, 7, 8, 511, 512, 2047, 2048, T // 2 - 1, T // 2, T - 2, T - 1}
+                           | set(g.integers(0, T, size=36).tolist())), dtype=np.int64)
+    qs = np.concatenate([WL.qI_lowrank(w, int(t), int(t) + 1) for t in rows]).reshape(len(rows), Hi, di)
+    idx_o, S = O.indexer_topk(qs, wt[rows], K, rows, m, k)
+    ig = idx.cpu().numpy()[rows]
+    same = check_topk(ig, idx_o, S, O.n_vis(rows, m), k)
+    assert same >= len(rows) - 2
+    # selected scores match the oracle's values of the same entries
+    scg = sc.cpu().numpy()[rows]
+    for r in range(len(rows)):
+        sel = ig[r][ig[r] >= 0]
+        np.testing.assert_allclose(scg[r][:len(sel)], S[r, sel], rtol=1e-4, atol=1e-3)
+
+
+def test_csa_prefill_64k_attention_sampled(C, csa64k):
+    w = csa64k
+    T, c, H, m, k, W = w.T, w.c, w.H, w.m, w.k, w.W
+    n = T // m
+    q = torch.empty((T, H * c), dtype=torch.bfloat16, device="cuda")
+    for r0 in range(0, T, 256):
+        q[r0:r0 + 256].copy_(torch.from_numpy(WL.draw(w, "q", r0, r0 + 256)).to(torch.bfloat16))
+    X = _fill(w, "X", T, c)
+    KVc = WL.draw(w, "KV", 0, n)
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    rows = _sample_rows(T, m, 13, n_random=96, head=64)
+    idx_all = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    for r0 in range(0, T, 4096):
+        idx_all[r0:r0 + 4096].copy_(torch.from_numpy(WL.random_topk_idx(w.seed, T, m, k, n, rows=range(r0, r0 + 4096))))
+    o = C.hybrid_attn_prefill(q.view(T, H, c), X, dev(KVc, "bf16"), dev(sink), 1.0, m, W, idx=idx_all)
+    torch.cuda.synchronize()
+    idx_rows = WL.random_topk_idx(w.seed, T, m, k, n, rows=rows)
+    idx_full = np.full((T, k), -1, np.int32)
+    idx_full[rows] = idx_rows
+    qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1)[0] for t in rows]).reshape(len(rows), H, c)
+    o_ref, _ = O.hybrid_attn_prefill(qs, WL.draw(w, "X", 0, T), KVc, sink, 1.0, m, W, idx=idx_full, rows=rows)
+    err = row_rel_err(host(o.view(T, H, c)[torch.from_numpy(rows).cuda()]), o_ref)
+    assert err.max() < 2e-2, err.max()
+
+
+def test_csa_decode_1m_full(C):
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, H, c, Hi, di, W, m, k = w.B, w.H, w.c, w.H_I, w.d_I, w.W, w.m, w.k
+    t = w.T
+    nv = (t + 1) // m
+    comp = C.KvRows.empty(Bn * nv, c, w.rope, "cuda")
+    keys = C.Fp4Rows.empty(Bn * nv, di, "cuda")
+    chunk = 32768
+    for b in range(Bn):
+        for r0 in range(0, nv, chunk):
+            r1 = min(nv, r0 + chunk)
+            sl = slice(b * nv + r0, b * nv + r1)
+            C.csa_quantize_kv(torch.from_numpy(WL.draw(w, "KV", r0, r1, seq=b)).cuda(),
+                              C.KvRows(comp.fp8[sl], comp.rope[sl], comp.scale[sl]))
+            C.csa_quantize_fp4(torch.from_numpy(WL.draw(w, "KI", r0, r1, seq=b)).cuda(),
+                               C.Fp4Rows(keys.codes[sl], keys.scales[sl]))
+    win = np.concatenate([WL.draw(w, "WIN", 0, W, seq=b) for b in range(Bn)])
+    wkv = C.KvRows.empty(Bn * W, c, w.rope, "cuda")
+    C.csa_quantize_kv(torch.from_numpy(win).cuda(), wkv)
+    q = np.stack([WL.draw(w, "q", 0, 1, seq=b).reshape(H, c) for b in range(Bn)])
+    qx = np.concatenate([WL.draw(w, "qI", 0, 1, seq=b).reshape(Hi, di) for b in range(Bn)])
+    wt = np.concatenate([WL.draw(w, "w", 0, 1, seq=b) for b in range(Bn)])
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    q4 = C.Fp4Rows.empty(Bn * Hi, di, "cuda")
+    C.csa_quantize_fp4(torch.from_numpy(qx).cuda(), q4)
+    pos = torch.full((Bn,), t, dtype=torch.int64, device="cuda")
+    off = torch.arange(Bn, dtype=torch.int64, device="cuda") * nv
+    idx = C.indexer_topk(q4, dev(wt), keys, m, k, max_nvis=nv, q_pos=pos, key_off=off)
+    o = C.hybrid_attn_decode(dev(q, "bf16"), comp, off, pos, wkv, torch.full((Bn,), W, dtype=torch.int32, device="cuda"),
+                             dev(sink), 1.0, m, W, max_nvis=nv, idx=idx)
+    torch.cuda.synchronize()
+    ig = idx.cpu().numpy()
+    og = host(o)
+    assert C.csa_device_error() == 0
+    # oracle, one sequence at a time
+    qc, qs_ = O.quant_fp4(qx)
+    Qd = O.dequant_fp4(qc, qs_).reshape(Bn, Hi, di)
+    wf, wr, wsc = O.quant_kv(win)
+    winrows = O.dequant_kv(wf, wr, wsc)
+    same_rows = 0
+    for b in range(Bn):
+        kb = np.concatenate([WL.draw(w, "KI", r0, min(nv, r0 + chunk), seq=b) for r0 in range(0, nv, chunk)])
+        kc, ks = O.quant_fp4(kb)
+        Kd = O.dequant_fp4(kc, ks)
+        del kb
+        idx_o, S = O.indexer_topk(Qd[b:b + 1], wt[b:b + 1], Kd, np.array([t]), m, k)
+        del Kd
+        same_rows += check_topk(ig[b:b + 1], idx_o, S, [nv], k)
+        if set(ig[b].tolist()) != set(idx_o[0].tolist()):
+            continue
+        sel = np.sort(idx_o[0])
+        rows_kv = np.concatenate([WL.draw(w, "KV", int(s), int(s) + 1, seq=b) for s in sel])
+        f8, rb, sc = O.quant_kv(rows_kv)
+        comp_sel = O.dequant_kv(f8, rb, sc)
+        remap = {int(s): j for j, s in enumerate(sel)}
+        idx_local = np.array([[remap[int(s)] for s in idx_o[0]]], np.int32)
+        o_ref, _ = O.hybrid_attn_decode(WL.on_grid(q[b:b + 1], "bf16"), comp_sel, [0], [t],
+                                        winrows[b * W:(b + 1) * W], [W], sink, 1.0, m, W, idx=idx_local)
+        err = row_rel_err(og[b:b + 1], o_ref)
+        assert err.max() < 2e-2, (b, err.max())
+    assert same_rows >= Bn - 1
