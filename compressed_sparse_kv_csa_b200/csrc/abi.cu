@@ -24,6 +24,9 @@ int *dev_error_word()
 cudaError_t launch_attn_prefill_generic(const PrefillArgs &a, cudaStream_t st);
 cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled);
 cudaError_t launch_indexer_scores_tc(const IndexerArgs &a, cudaStream_t st, bool *handled);
+size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k);
+bool decode_indexer_eligible(const IndexerArgs &a);
+cudaError_t launch_indexer_decode(const IndexerArgs &a, void *ws, cudaStream_t st);
 } // namespace csa
 
 using namespace csa;
@@ -153,9 +156,10 @@ int csa_quantize_fp4(const void *x, int32_t in_dtype, int64_t n, int32_t d,
 
 size_t indexer_topk_workspace_size(int64_t Nq, int64_t max_nvis, int32_t k)
 {
-    (void)k;
-    if (Nq < 0 || max_nvis < 0) return 0;
-    return round_up((size_t)Nq * (size_t)score_ld(max_nvis) * sizeof(float)) + kAlign;
+    if (Nq < 0 || max_nvis < 0 || k < 0) return 0;
+    const size_t dense = round_up((size_t)Nq * (size_t)score_ld(max_nvis) * sizeof(float)) + kAlign;
+    const size_t decode = round_up(decode_indexer_workspace(Nq, max_nvis, k)) + kAlign;
+    return dense > decode ? dense : decode;
 }
 
 int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
@@ -201,6 +205,8 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
     a.score_out = score_out;
     a.err = dev_error_word();
     if (Nq == 0) return CSA_OK;
+    if (decode_indexer_eligible(a)) // FP4, 64 x 128: fused tensor-core scan + chunked top-k
+        return status_of(launch_indexer_decode(a, reinterpret_cast<void *>(base), S(stream)));
     bool handled = false;
     cudaError_t e = launch_indexer_scores_tc(a, S(stream), &handled);
     if (!handled) e = launch_indexer_scores(a, S(stream));

@@ -52,9 +52,10 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0;
             __syncthreads();
-            for (int64_t s = tid; s < nv; s += TK_THREADS) {
-                const uint32_t key = float_key(S[s]);
-                if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+            for (int64_t b0 = 0; b0 < nv; b0 += TK_THREADS) { // warp-uniform trip count
+                const int64_t s = b0 + tid;
+                const uint32_t key = s < nv ? float_key(S[s]) : 0u;
+                hist_add(hist, (int)((key >> shift) & 255), s < nv && (key & pmask) == prefix);
             }
             __syncthreads();
             if (tid == 0) {

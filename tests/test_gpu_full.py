@@ -205,7 +205,7 @@ def test_csa_decode_1m_full(C):
         if set(ig[b].tolist()) != set(idx_o[0].tolist()):
             continue
         sel = np.sort(idx_o[0])
-        rows_kv = np.concatenate([WL.draw(w, "KV", int(s), int(s) + 1, seq=b) for s in sel])
+        rows_kv = WL.draw(w, "KV", 0, nv, seq=b)[sel]
         f8, rb, sc = O.quant_kv(rows_kv)
         comp_sel = O.dequant_kv(f8, rb, sc)
         remap = {int(s): j for j, s in enumerate(sel)}

@@ -172,7 +172,7 @@ def test_indexer_topk_fp4_decode_batches(C):
     """FP4 queries and keys with per-sequence key offsets and positions (decode layout)."""
     w = WL.WORKLOADS["csa_decode_1m"]
     Bn, H, d, k, m = 3, 64, 128, 1024, 4
-    pos = np.array([4 * 3000 + 2, 40001, 4 * 1500 - 1], np.int64)
+    pos = np.array([4 * 3001 + 2, 4 * 17001 + 1, 4 * 1500 - 1], np.int64)  # odd key offsets
     nv = O.n_vis(pos, m)
     off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
     keys = np.concatenate([WL.draw(w, "KI", 0, int(n), seq=b) for b, n in enumerate(nv)])
@@ -190,6 +190,27 @@ def test_indexer_topk_fp4_decode_batches(C):
     idx = C.indexer_topk(q4, dev(wt), k4, m, k, max_nvis=int(nv.max()),
                          q_pos=torch.from_numpy(pos).cuda(), key_off=torch.from_numpy(off).cuda())
     assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
+
+
+def test_fp4_decode_topk_ties_across_chunks(C):
+    """All scores equal (q = 0): every query keeps the lowest k entries, which requires the
+    per-chunk selections and their merge to break ties by entry index."""
+    Bn, H, d, k = 2, 64, 128, 1024
+    nv = np.array([40000, 700], np.int64)
+    off = np.array([5, 40005], np.int64)
+    g = np.random.default_rng(9)
+    keys = g.standard_normal((int(off[-1] + nv[-1]), d)).astype(np.float32)
+    k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
+    C.csa_quantize_fp4(dev(keys), k4)
+    q4 = C.Fp4Rows.empty(Bn * H, d, "cuda")
+    C.csa_quantize_fp4(torch.zeros((Bn * H, d), device="cuda"), q4)
+    sc = torch.empty((Bn, k), dtype=torch.float32, device="cuda")
+    idx = C.indexer_topk(q4, torch.ones((Bn, H), device="cuda"), k4, 4, k, max_nvis=int(nv.max()),
+                         q_pos=torch.from_numpy(nv * 4 - 1).cuda(), key_off=torch.from_numpy(off).cuda(), score_out=sc)
+    ig = idx.cpu().numpy()
+    assert list(ig[0]) == list(range(k))
+    assert list(ig[1]) == list(range(700)) + [-1] * (k - 700)
+    assert np.all(sc.cpu().numpy()[idx.cpu().numpy() >= 0] == 0.0)
 
 
 def test_topk_ties_short_lists_and_scores(C):
