@@ -27,6 +27,10 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs &a, cudaStream_t st, bool
 size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k);
 bool decode_indexer_eligible(const IndexerArgs &a);
 cudaError_t launch_indexer_decode(const IndexerArgs &a, void *ws, cudaStream_t st);
+int decode_tc_chunks(int64_t max_keys);
+bool decode_attn_tc_eligible(const DecodeArgs &a);
+cudaError_t launch_attn_decode_tc(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st);
 } // namespace csa
 
 using namespace csa;
@@ -49,7 +53,7 @@ bool kv_rows_ok(const csa_kv_rows *kv, int64_t n_min, int32_t c)
 bool fp4_rows_ok(const csa_fp4_rows *f, int64_t n_min, int32_t d)
 {
     if (!f || !f->codes || !f->scales || f->d != d || f->n < n_min || (d % 32)) return false;
-    return aligned16(f->codes);
+    return aligned16(f->codes) && (reinterpret_cast<uintptr_t>(f->scales) & 3u) == 0;
 }
 
 KvRowsDev to_dev(const csa_kv_rows &k) { return KvRowsDev{k.fp8, k.rope, k.scale, k.n, k.c, k.rope_dims}; }
@@ -245,6 +249,8 @@ size_t hybrid_attn_decode_workspace_size(int32_t B, int32_t H, int32_t c, int32_
     if (max_keys > (int64_t)1 << 30) return 0;
     int nc, ch;
     decode_plan(B, H, c, (int)(max_keys > 0 ? max_keys : 1), &nc, &ch);
+    const int nc_tc = decode_tc_chunks(max_keys > 0 ? max_keys : 1); // tensor-core path: 128-key chunks
+    if (nc_tc > nc) nc = nc_tc;
     return round_up((size_t)B * nc * H * (c + 2) * sizeof(float)) + kAlign;
 }
 
@@ -288,9 +294,16 @@ int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *co
     a.lse = lse;
     a.err = dev_error_word();
     const int64_t max_keys = (int64_t)W + (idx ? k : max_nvis);
-    decode_plan(B, H, c, (int)max_keys, &a.n_chunks, &a.chunk);
     uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + kAlign - 1) / kAlign * kAlign;
     a.part = reinterpret_cast<float *>(base);
+    a.n_chunks = decode_tc_chunks(max_keys);
+    a.chunk = 128;
+    if (decode_attn_tc_eligible(a)) { // 64 heads x 512 channels: tcgen05 split-K + merge
+        cudaError_t e = launch_attn_decode_tc(a, S(stream));
+        if (e != cudaSuccess) return CSA_ERR_CUDA;
+        return status_of(launch_decode_merge(a, S(stream)));
+    }
+    decode_plan(B, H, c, (int)max_keys, &a.n_chunks, &a.chunk);
     return status_of(launch_attn_decode(a, S(stream)));
 }
 

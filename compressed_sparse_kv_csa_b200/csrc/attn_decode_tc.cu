@@ -1,0 +1,284 @@
+// attn_decode_tc.cu -- hybrid MQA decode attention on tcgen05 for 64 heads x 512 channels over the
+// mixed FP8/BF16 caches: one new token per sequence, split-K over 128-key chunks of its key list.
+//
+// Method: "DeepSeek-V4: Towards Highly Efficient Million-Token Context Intelligence" paper notes,
+// Sec. 2.3 step 3 (shared-KV multi-query attention, the key vector is also the value vector) and
+// Sec. 2.4 Attention.forward listing (window keys and selected / all visible compressed keys,
+// concatenated); KV cache with BF16 RoPE dims and FP8 for the rest ("Mind Observatory: Uncovering
+// the technical ledger of DeepSeek-V4"); the per-head sink is folded in by the merge kernel.
+//
+// Grid = (chunks of 128 keys, sequences).  Each CTA:
+//   1. stages q [64 x 512] (bf16) and gathers its 128 key rows -- window rows first, then the
+//      top-k (CSA) or visible (HCA) compressed rows -- dequantising the FP8 part (code x row scale)
+//      to bf16 next to the BF16 RoPE part, all in 128-byte-swizzled shared memory;
+//   2. one thread issues S = Q K^T (tcgen05 M=64, N=128, K=512) into TMEM;
+//   3. 4 warps take the softmax of their 16 heads over the chunk (lanes l and l+16 split the
+//      keys), writing P (bf16) to shared memory and (max, sum) to the workspace;
+//   4. O = P V (two M=64 x N=256 x K=128 MMAs, V = the same tile read MN-major) into TMEM, and
+//      the unnormalised O rows go to the workspace for the split-K merge.
+#include "common.cuh"
+#include "tc_common.cuh"
+
+namespace csa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kH = 64, kC = 512, kKT = 128;
+constexpr int kThreads = 8 * 32 + 32; // 8 warps + 1 MMA / TMEM warp
+constexpr int kMmaWarp = 8;
+constexpr uint32_t OFF_Q = 0;        // 8 sub-tiles [64 x 128 B]   64 KB
+constexpr uint32_t OFF_K = 65536;    // 8 sub-tiles [128 x 128 B]  128 KB
+constexpr uint32_t OFF_P = 196608;   // 2 sub-tiles [64 x 128 B]   16 KB
+constexpr uint32_t OFF_VALID = 212992; // 128 flags
+constexpr uint32_t OFF_BAR = OFF_VALID + 512;
+constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
+constexpr uint32_t SMEM_ALLOC = OFF_TMEM + 64 + 1024;
+constexpr uint32_t TMEM_O = 16u << 16;
+constexpr uint32_t kColS = 256;
+constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(64, 256, false, true);
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ void sts4(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pk_bf16(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// 8 FP8 E4M3 codes (one uint2) times the row scale -> 8 bf16 (one uint4)
+__device__ __forceinline__ uint4 fp8x8_to_bf16(uint2 c, float s)
+{
+    const uint32_t w[2] = {c.x, c.y};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffff), __NV_E4M3);
+        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
+        const float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+        o[2 * i] = pk_bf16(a.x * s, a.y * s);
+        o[2 * i + 1] = pk_bf16(b.x * s, b.y * s);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (base - raw);
+    const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sP = base + OFF_P;
+    const uint32_t bar_s = base + OFF_BAR, bar_o = base + OFF_BAR + 8, bar_f = base + OFF_BAR + 16;
+    int *valid = reinterpret_cast<int *>(sp + OFF_VALID);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.y, chunk = blockIdx.x;
+    const int n_win = a.win_len[b] < 0 ? 0 : (a.win_len[b] > a.W ? a.W : a.win_len[b]);
+    int64_t n_cmp;
+    if (a.idx) n_cmp = a.k;
+    else {
+        n_cmp = (a.pos[b] + 1) / a.m;
+        if (n_cmp > a.max_nvis) n_cmp = a.max_nvis;
+        if (n_cmp < 0) n_cmp = 0;
+    }
+    const int64_t n_keys = n_win + n_cmp;
+    const int64_t j0 = (int64_t)chunk * kKT;
+    float *part = a.part + ((int64_t)b * a.n_chunks + chunk) * kH * (kC + 2);
+    if (j0 >= n_keys) { // empty chunk: a neutral partial (CTA-uniform exit)
+        for (int h = tid; h < kH; h += kThreads) {
+            part[(int64_t)h * (kC + 2)] = -INFINITY;
+            part[(int64_t)h * (kC + 2) + 1] = 0.f;
+        }
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        mbar_init(bar_f, 1);
+        mbar_init_fence();
+    }
+    if (warp == kMmaWarp) tmem_alloc(base + OFF_TMEM, 512);
+
+    // ---- stage q and gather the chunk's key rows (all 288 threads)
+    for (int e = tid; e < kH * (kC / 8); e += kThreads) {
+        const int h = e >> 6, cc = e & 63;
+        const uint4 v = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + h) * kC + 8 * cc);
+        sts4(sQ + (uint32_t)(cc >> 3) * 8192u + sw128_off(h, (cc & 7) * 8), v);
+    }
+    const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
+    for (int e = tid; e < kKT * (kC / 8); e += kThreads) {
+        const int jj = e >> 6, cc = e & 63; // key slot, 8-channel chunk
+        const int64_t j = j0 + jj;
+        const KvRowsDev *kv = nullptr;
+        int64_t row = -1;
+        if (j < n_keys && j < n_win) {
+            kv = &a.win;
+            row = (int64_t)b * a.W + j;
+        } else if (j < n_keys) {
+            const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
+            if (s >= 0) {
+                const int64_t r = a.comp_off[b] + s;
+                if (r >= 0 && r < a.comp.n) {
+                    kv = &a.comp;
+                    row = r;
+                } else if (cc == 0) {
+                    flag_error(a.err, CSA_DEVERR_INDEX);
+                }
+            }
+        }
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (kv) {
+            const int ch = 8 * cc;
+            if (ch < cn) v = fp8x8_to_bf16(*reinterpret_cast<const uint2 *>(kv->fp8 + row * cn + ch), kv->scale[row]);
+            else v = *reinterpret_cast<const uint4 *>(kv->rope + row * kv->rope_dims + (ch - cn));
+        }
+        sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
+        if (cc == 0) valid[jj] = kv ? 1 : 0;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + OFF_TMEM);
+    bool ok = true;
+
+    if (warp == kMmaWarp && lane == 0) { // S = Q K^T
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + kColS, sdesc_sw128(sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024),
+                         sdesc_sw128(sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024), IDESC_S, (s | kk) != 0);
+        mma_commit(bar_s);
+    }
+    const bool upper = lane < 16;
+    const int row = 16 * (warp & 3) + (lane & 15);
+    if (warp < 4) { // softmax of the chunk: lane l keys 0-63, lane l+16 keys 64-127 of head `row`
+        const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s, 0));
+        if (ok) {
+            tc_fence_after();
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32(tw + kColS, r0);
+            tmem_ld32(tw + kColS + 32, r1);
+            tmem_ld32(tw + kColS + 64, r2);
+            tmem_ld32(tw + kColS + 96, r3);
+            tmem_ld_wait();
+            float sv[64];
+            const int kb = upper ? 0 : 64;
+            const float sl2 = a.scale * kLog2e;
+            float mt = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
+                const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
+                float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
+                s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
+                s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
+                sv[e] = s0;
+                sv[32 + e] = s1;
+                mt = fmaxf(mt, fmaxf(s0, s1));
+            }
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+            float ls = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                const float p = (mt == -INFINITY) ? 0.f : ex2(sv[e] - mt);
+                sv[e] = p;
+                ls += p;
+            }
+            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+            const uint32_t psub = sP + (uint32_t)(kb >> 6) * 8192u;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                sts4(psub + sw128_off(row, 8 * g),
+                     make_uint4(pk_bf16(sv[8 * g], sv[8 * g + 1]), pk_bf16(sv[8 * g + 2], sv[8 * g + 3]),
+                                pk_bf16(sv[8 * g + 4], sv[8 * g + 5]), pk_bf16(sv[8 * g + 6], sv[8 * g + 7])));
+            if (upper) {
+                part[(int64_t)row * (kC + 2)] = (mt == -INFINITY) ? -INFINITY : mt * kLn2; // natural-log max
+                part[(int64_t)row * (kC + 2) + 1] = ls;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+    }
+    __syncthreads();
+    ok = __syncthreads_and(ok);
+    if (warp == kMmaWarp && lane == 0 && ok) { // O = P V
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16(h ? tmem : tmem + TMEM_O,
+                         sdesc_sw128(sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024),
+                         sdesc_sw128(sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024), IDESC_PV, kk > 0);
+        mma_commit(bar_o);
+    }
+    if (warp < 4 && ok) { // unnormalised O rows -> workspace (lane l: channels 256-511, l+16: 0-255)
+        const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+        if (__all_sync(0xffffffffu, mbar_wait(bar_o, 0))) {
+            tc_fence_after();
+            float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tw + 32u * c, r);
+                tmem_ld_wait();
+                // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
+                // 8-byte stores are the widest that are aligned for every row
+#pragma unroll
+                for (int g = 0; g < 16; ++g)
+                    *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
+                        make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
+            }
+        } else {
+            ok = false;
+        }
+        tc_fence_before();
+    }
+    if (!ok && tid == 0) flag_error(a.err, CSA_DEVERR_TIMEOUT);
+    if (warp == kMmaWarp && lane == 0) {
+        mma_commit(bar_f);
+        if (!mbar_wait(bar_f, 0)) flag_error(a.err, CSA_DEVERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+} // namespace
+
+int decode_tc_chunks(int64_t max_keys) { return (int)((max_keys + kKT - 1) / kKT); }
+
+bool decode_attn_tc_eligible(const DecodeArgs &a)
+{
+    return a.H == kH && a.c == kC && a.comp.rope_dims == a.win.rope_dims && (kC - a.comp.rope_dims) % 8 == 0 &&
+           a.comp.rope_dims % 8 == 0 && a.n_chunks <= 1024;
+}
+
+cudaError_t launch_attn_decode_tc(const DecodeArgs &a, cudaStream_t st)
+{
+    cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    decode_attn_tc_kernel<<<dim3((unsigned)a.n_chunks, (unsigned)a.B), kThreads, SMEM_ALLOC, st>>>(a);
+    return cudaGetLastError();
+}
+
+} // namespace csa

@@ -201,6 +201,38 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
     const int64_t c1 = (c0 + a.chunk) < n_keys ? (c0 + a.chunk) : n_keys;
     const int64_t cbase = a.comp_off[b];
 
+    // gather key rows j0 .. j0+KT-1 of this sequence's list (dequantised to fp32) into the tile
+    auto stage = [&](int64_t j0) {
+        for (int e = threadIdx.x; e < KT * (C / 4); e += NWARP * 32) {
+            const int jj = e / (C / 4), ch = (e % (C / 4)) * 4;
+            const int64_t j = j0 + jj;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            int ok = 0;
+            if (j < c1 && j < n_win) { // window row (rows b*W .. b*W+W-1 exist: checked on host)
+                v = kv_row4(a.win, (int64_t)b * a.W + j, ch);
+                ok = 1;
+            } else if (j < c1) {        // compressed entry
+                const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
+                if (s >= 0) {
+                    const int64_t row = cbase + s;
+                    if (row >= 0 && row < a.comp.n) {
+                        v = kv_row4(a.comp, row, ch);
+                        ok = 1;
+                    } else if (ch == 0) {
+                        flag_error(a.err, CSA_DEVERR_INDEX);
+                    }
+                }
+            }
+            *reinterpret_cast<float4 *>(kt + jj * C + ch) = v;
+            if (ch == 0) kvalid[jj] = ok;
+        }
+    };
+    // a chunk of at most one tile is staged once for all head passes
+    const bool single = (c1 - c0) <= KT;
+    if (single) {
+        stage(c0);
+        __syncthreads();
+    }
     for (int h0 = 0; h0 < H; h0 += NWARP) {
         const int h = h0 + warp;
         const bool hact = h < H;
@@ -214,31 +246,11 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
             qv[i] = hact ? bf16_to_f32(a.q[((int64_t)b * H + h) * C + lane + 32 * i]) : 0.f;
         }
         for (int64_t j0 = c0; j0 < c1; j0 += KT) {
-            __syncthreads();
-            for (int e = threadIdx.x; e < KT * (C / 4); e += NWARP * 32) {
-                const int jj = e / (C / 4), ch = (e % (C / 4)) * 4;
-                const int64_t j = j0 + jj;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                int ok = 0;
-                if (j < c1 && j < n_win) { // window row (rows b*W .. b*W+W-1 exist: checked on host)
-                    v = kv_row4(a.win, (int64_t)b * a.W + j, ch);
-                    ok = 1;
-                } else if (j < c1) {        // compressed entry
-                    const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
-                    if (s >= 0) {
-                        const int64_t row = cbase + s;
-                        if (row >= 0 && row < a.comp.n) {
-                            v = kv_row4(a.comp, row, ch);
-                            ok = 1;
-                        } else if (ch == 0) {
-                            flag_error(a.err, CSA_DEVERR_INDEX);
-                        }
-                    }
-                }
-                *reinterpret_cast<float4 *>(kt + jj * C + ch) = v;
-                if (ch == 0) kvalid[jj] = ok;
+            if (!single) {
+                __syncthreads();
+                stage(j0);
+                __syncthreads();
             }
-            __syncthreads();
             if (hact) {
                 const int nj = (int)((c1 - j0) < KT ? (c1 - j0) : KT);
                 for (int jj = 0; jj < nj; ++jj)
@@ -254,35 +266,45 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
     }
 }
 
+// One CTA per (sequence, head): fold the chunks' (max, sum, unnormalised output) and the sink.
+// The per-chunk weights e^{m_j - m} / denominator are computed once into shared memory.
+constexpr int kMaxMergeChunks = 1024;
+
 __global__ void decode_merge_kernel(DecodeArgs a)
 {
+    __shared__ float fac[kMaxMergeChunks];
+    __shared__ float s_m, s_l;
     const int bh = blockIdx.x; // b * H + h
     const int b = bh / a.H, h = bh % a.H;
-    const int C = a.c;
-    const float *p0 = a.part + ((int64_t)b * a.n_chunks * a.H + h) * (C + 2);
+    const int C = a.c, nc = a.n_chunks;
+    const float *p0 = a.part + ((int64_t)b * nc * a.H + h) * (C + 2);
     const int64_t cstride = (int64_t)a.H * (C + 2);
-    float mt = a.sink[h];
-    for (int j = 0; j < a.n_chunks; ++j) mt = fmaxf(mt, p0[j * cstride]);
-    float lt = 0.f;
-    if (mt > -INFINITY) {
-        lt = __expf(a.sink[h] - mt);
-        for (int j = 0; j < a.n_chunks; ++j) {
+    if (threadIdx.x < 32) {
+        float mt = a.sink[h];
+        for (int j = threadIdx.x; j < nc; j += 32) mt = fmaxf(mt, p0[j * cstride]);
+        mt = warp_max(mt);
+        float lt = 0.f;
+        for (int j = threadIdx.x; j < nc; j += 32) {
             const float mj = p0[j * cstride];
-            if (mj > -INFINITY) lt += p0[j * cstride + 1] * __expf(mj - mt);
+            lt += (mj > -INFINITY) ? p0[j * cstride + 1] * __expf(mj - mt) : 0.f;
         }
+        lt = warp_sum(lt);
+        if (mt > -INFINITY) lt += __expf(a.sink[h] - mt);
+        const float inv = (mt > -INFINITY && lt > 0.f) ? 1.f / lt : 0.f;
+        for (int j = threadIdx.x; j < nc; j += 32) {
+            const float mj = p0[j * cstride];
+            fac[j] = (mj > -INFINITY) ? __expf(mj - mt) * inv : 0.f;
+        }
+        if (threadIdx.x == 0) { s_m = mt; s_l = lt; }
     }
+    __syncthreads();
     for (int ch = threadIdx.x; ch < C; ch += blockDim.x) {
         float acc = 0.f;
-        if (mt > -INFINITY) {
-            for (int j = 0; j < a.n_chunks; ++j) {
-                const float mj = p0[j * cstride];
-                if (mj > -INFINITY) acc += p0[j * cstride + 2 + ch] * __expf(mj - mt);
-            }
-            acc /= lt;
-        }
+        for (int j = 0; j < nc; ++j) // chunks without keys carry weight 0 and unwritten rows
+            if (fac[j] != 0.f) acc = fmaf(p0[j * cstride + 2 + ch], fac[j], acc);
         a.o[(int64_t)bh * C + ch] = f32_to_bf16_bits(acc);
     }
-    if (a.lse && threadIdx.x == 0) a.lse[bh] = (mt > -INFINITY) ? mt + __logf(lt) : -INFINITY;
+    if (a.lse && threadIdx.x == 0) a.lse[bh] = (s_m > -INFINITY) ? s_m + __logf(s_l) : -INFINITY;
 }
 
 template <int CPL>
@@ -322,6 +344,13 @@ void decode_plan(int B, int H, int c, int max_keys, int *n_chunks, int *chunk)
     *n_chunks = (max_keys + ch - 1) / ch;
     if (*n_chunks < 1) *n_chunks = 1;
     *chunk = ch;
+}
+
+cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st)
+{
+    if (a.n_chunks > kMaxMergeChunks) return cudaErrorInvalidValue;
+    decode_merge_kernel<<<(unsigned)(a.B * a.H), 128, 0, st>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_attn_decode(const DecodeArgs &a, cudaStream_t st)

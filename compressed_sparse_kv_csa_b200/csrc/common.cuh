@@ -133,17 +133,6 @@ __device__ __forceinline__ float key_float(uint32_t k)
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Warp-aggregated histogram increment: lanes with the same bin add once through their lowest
-// lane (radix-select histograms are heavily skewed, so plain per-lane atomics serialise).  Must
-// be called by all 32 lanes; inactive lanes pass active = false.
-__device__ __forceinline__ void hist_add(int *hist, int bin, bool active)
-{
-    const int lane = threadIdx.x & 31;
-    const int key = active ? bin : (1 << 20) + lane; // inactive lanes form singleton groups
-    const unsigned grp = __match_any_sync(0xffffffffu, key);
-    if (active && (__ffs(grp) - 1) == lane) atomicAdd(&hist[bin], __popc(grp));
-}
-
 __device__ __forceinline__ float warp_sum(float v)
 {
 #pragma unroll

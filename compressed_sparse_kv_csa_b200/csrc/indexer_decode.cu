@@ -6,10 +6,11 @@
 // s < N_vis(t), then the k best entries); the indexer's QK path runs in FP4 E2M1 with 32-element
 // block scales (itsolotime.com Q&A essay on DeepSeek-V4, Question 4; "technical ledger" page).
 //
-// Kernel 1 (grid = key chunks x queries): each CTA streams its chunk of up to 16,384 FP4 keys
+// Kernel 1 (grid = key chunks x queries, about one CTA per SM): each CTA streams its chunk of up
+// to 16,384 FP4 keys
 //   * one lane issues bulk copies of 128-key tiles (8 KB of E2M1 codes + 512 B of E8M0 scales)
 //     into a 4-stage ring;
-//   * 4 converter warps turn a tile into f16 in the 128-byte-swizzled MMA layout with the
+//   * 8 converter warps turn a tile into f16 in the 128-byte-swizzled MMA layout with the
 //     hardware E2M1x2 -> f16x2 conversion, folding each block's power-of-two scale in with one
 //     f16x2 multiply (exact while the block's scale exponent lies in [-23, 13]);
 //   * one lane issues tcgen05 M=128 (keys) x N=64 (heads) x K=128 f16 MMAs against the query,
@@ -24,6 +25,7 @@
 // Every wait is bounded (%globaltimer); a timeout sets CSA_DEVERR_TIMEOUT and the CTA returns.
 #include "common.cuh"
 #include "tc_common.cuh"
+#include "select.cuh"
 
 namespace csa {
 
@@ -32,9 +34,10 @@ namespace {
 using namespace tc;
 
 constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 4;
-constexpr int kChunk = 16384;                 // keys per CTA
-constexpr int kThreads = 10 * 32;
-constexpr int kProdWarp = 0, kConvWarp0 = 1, kEpiWarp0 = 5, kMmaWarp = 9;
+constexpr int kChunk = 16384;                 // most keys per CTA (scores stay in shared memory)
+constexpr int kConvWarps = 8;
+constexpr int kProdWarp = 0, kConvWarp0 = 1, kEpiWarp0 = kConvWarp0 + kConvWarps, kMmaWarp = kEpiWarp0 + 4;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kStageCodes = kKT * kDI / 2;     // 8192 B
 constexpr uint32_t kStageBytes = kStageCodes + kKT * (kDI / 32); // + 512 B scales
 
@@ -43,8 +46,8 @@ constexpr uint32_t OFF_A = 65536;                            // 2 x [128 x 128] 
 constexpr uint32_t OFF_B = OFF_A + 65536;                    // [64 x 128] f16 = 16 KB
 constexpr uint32_t OFF_ST = OFF_B + 16384;                   // 4 x 8704 B staging
 constexpr uint32_t OFF_W = OFF_ST + kStages * kStageBytes;   // w [64] fp32
-constexpr uint32_t OFF_HIST = OFF_W + 256;                   // 256 ints
-constexpr uint32_t OFF_MISC = OFF_HIST + 1024;               // counters
+constexpr uint32_t OFF_HIST = OFF_W + 256;                   // selection scratch (< 2 KB)
+constexpr uint32_t OFF_MISC = OFF_HIST + 2048;               // counters
 constexpr uint32_t OFF_BAR = OFF_MISC + 256;
 constexpr uint32_t OFF_TMEM = OFF_BAR + 256;
 constexpr uint32_t SMEM_USED = OFF_TMEM + 16;
@@ -138,7 +141,7 @@ __device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity)
 // ------------------------------------------------------------------------------------------
 template <int NT>
 __device__ void chunk_topk(uint32_t sc_base, int n, int k, int64_t entry0, unsigned long long *out, int *out_count,
-                           int *hist, int *misc)
+                           SelectSmem<uint32_t> *sel, int *misc)
 {
     const int tid = threadIdx.x;
     auto score_key = [&](int i) {
@@ -154,34 +157,10 @@ __device__ void chunk_topk(uint32_t sc_base, int n, int k, int64_t entry0, unsig
         if (tid == 0) *out_count = n;
         return;
     }
-    uint32_t prefix = 0, pmask = 0;
-    int rem = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += NT) hist[i] = 0;
-        __syncthreads();
-        for (int b0 = 0; b0 < n; b0 += NT) { // warp-uniform trip count
-            const int i = b0 + tid;
-            const uint32_t key = i < n ? score_key(i) : 0u;
-            hist_add(hist, (int)((key >> shift) & 255), i < n && (key & pmask) == prefix);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int cum = 0, b = 255;
-            for (; b > 0; --b) {
-                if (cum + hist[b] >= rem) break;
-                cum += hist[b];
-            }
-            misc[0] = b;
-            misc[1] = rem - cum;
-        }
-        __syncthreads();
-        prefix |= (uint32_t)misc[0] << shift;
-        pmask |= 255u << shift;
-        rem = misc[1];
-        __syncthreads();
-    }
-    const uint32_t thr = prefix;
-    const int n_gt = k - rem;
+    uint32_t thr;
+    int n_gt;
+    block_kth<NT, uint32_t>(n, k, score_key, sel, thr, n_gt);
+    const int rem = k - n_gt;
     if (tid == 0) { misc[2] = 0; misc[3] = 0; }
     __syncthreads();
     for (int i = tid; i < n; i += NT) {
@@ -219,8 +198,8 @@ __device__ void chunk_topk(uint32_t sc_base, int n, int k, int64_t entry0, unsig
 // ------------------------------------------------------------------------------------------
 // kernel 1: FP4 key scan (tcgen05) + chunk top-k
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a, int n_slots, unsigned long long *cand,
-                                                                  int *cand_count)
+__global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a, int n_slots, int chunk,
+                                                                  unsigned long long *cand, int *cand_count)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -231,8 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     const int64_t r = blockIdx.y;
     const int slot = blockIdx.x;
     const int64_t nv = dec_nvis(a, r);
-    const int64_t c0 = (int64_t)slot * kChunk;
-    const int n = (int)(nv - c0 < kChunk ? (nv - c0 > 0 ? nv - c0 : 0) : kChunk);
+    const int64_t c0 = (int64_t)slot * chunk;
+    const int n = (int)(nv - c0 < chunk ? (nv - c0 > 0 ? nv - c0 : 0) : chunk);
     unsigned long long *out = cand + ((int64_t)r * n_slots + slot) * a.k;
     int *out_count = cand_count + r * n_slots + slot;
     if (n == 0) { // nothing visible in this chunk (CTA-uniform)
@@ -245,9 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     if (tid == 0) {
         for (int b = 0; b < NUM_BARS; ++b) {
             uint32_t cnt = 1;
-            if ((b >= B_STEMPTY && b < B_STEMPTY + kStages) || (b >= B_AFULL && b < B_AFULL + 2) ||
-                (b >= B_DEMPTY && b < B_DEMPTY + 2))
-                cnt = 128;
+            if ((b >= B_STEMPTY && b < B_STEMPTY + kStages) || (b >= B_AFULL && b < B_AFULL + 2))
+                cnt = 32 * kConvWarps;
+            if (b >= B_DEMPTY && b < B_DEMPTY + 2) cnt = 128;
+            if (b >= B_STFULL && b < B_STFULL + kStages) cnt = 1 + 32; // expect_tx arrive + 32 cp.async arrivals
             mbar_init(bar(b), cnt);
         }
         mbar_init_fence();
@@ -274,8 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
 
     bool ok = true;
     if (warp == kProdWarp) {
-        // codes: one bulk copy per tile (row0 * 64 bytes is always 16-byte aligned); scales: plain
-        // loads by the warp (a sequence's key offset need not be a multiple of 4 rows)
+        // codes: one bulk copy per tile (row0 * 64 bytes is always 16-byte aligned); scales: 4-byte
+        // cp.async per key row by the warp (a sequence's key offset need not be a multiple of 4
+        // rows), each lane arriving on the stage barrier when its copies land
         for (int i = 0; i < ntiles && ok; ++i) {
             const uint32_t st = i % kStages;
             if (i >= kStages && !wwait(bar(B_STEMPTY + st), ((i / kStages) - 1) & 1)) { ok = false; break; }
@@ -283,18 +264,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const int64_t rows_left = a.k4.n - row0; // never read past the key array
             const uint32_t nr = (uint32_t)(rows_left < kKT ? rows_left : kKT);
             const uint32_t dst = base + OFF_ST + st * kStageBytes;
-            for (uint32_t j = lane; j < nr * (kDI / 32); j += 32) {
-                const uint32_t v = a.k4.scales[row0 * (kDI / 32) + j];
-                asm volatile("st.shared.u8 [%0], %1;" ::"r"(dst + kStageCodes + j), "r"(v) : "memory");
-            }
-            __syncwarp();
+            for (uint32_t j = lane; j < nr; j += 32) // one 4-byte word of scales per key row
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + kStageCodes + 4u * j),
+                             "l"(a.k4.scales + (row0 + j) * (kDI / 32))
+                             : "memory");
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_STFULL + st)) : "memory");
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(B_STFULL + st), nr * (kDI / 2));
                 bulk_g2s(dst, a.k4.codes + row0 * (kDI / 2), nr * (kDI / 2), bar(B_STFULL + st));
             }
         }
     } else if (warp >= kConvWarp0 && warp < kEpiWarp0) {
-        const int ct = tid - 32 * kConvWarp0; // 0..127
+        const int ct = tid - 32 * kConvWarp0; // 0 .. 32*kConvWarps-1
         for (int i = 0; i < ntiles && ok; ++i) {
             const uint32_t st = i % kStages, ab = i & 1;
             if (!wwait(bar(B_STFULL + st), (i / kStages) & 1)) { ok = false; break; }
@@ -302,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const uint32_t stb = base + OFF_ST + st * kStageBytes;
             const int valid = n - i * kKT; // keys of this tile inside the chunk
 #pragma unroll 1
-            for (int p = 0; p < 4; ++p) {
-                const int key = (ct >> 2) + 32 * p, blk = ct & 3;
+            for (int p = 0; p < 512 / (32 * kConvWarps); ++p) { // 128 keys x 4 blocks per tile
+                const int key = (ct >> 2) + (8 * kConvWarps) * p, blk = ct & 3;
                 uint32_t v[16];
                 if (key < valid) {
                     uint4 codes;
@@ -374,8 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 128);
-    chunk_topk<kThreads>(base + OFF_SC, n, a.k, c0, out, out_count, reinterpret_cast<int *>(sp + OFF_HIST),
-                         reinterpret_cast<int *>(sp + OFF_MISC));
+    chunk_topk<kThreads>(base + OFF_SC, n, a.k, c0, out, out_count,
+                         reinterpret_cast<SelectSmem<uint32_t> *>(sp + OFF_HIST), reinterpret_cast<int *>(sp + OFF_MISC));
 }
 
 // ------------------------------------------------------------------------------------------
@@ -388,9 +369,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
                                                                      const int *cand_count)
 {
     extern __shared__ unsigned long long mv[];
-    __shared__ int hist[256];
-    __shared__ int s_bin, s_rem, s_cnt, s_off[64];
-    __shared__ unsigned long long s_prefix;
+    __shared__ SelectSmem<unsigned long long> msel;
+    __shared__ int s_cnt, s_off[64];
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
     const int k = a.k;
@@ -412,36 +392,13 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
     const int ke = total < k ? total : k;
     unsigned long long *sel = mv + total; // ke winners
     if (total > k) {
-        // radix select on the unique 64-bit keys: the k-th largest
-        unsigned long long prefix = 0, pmask = 0;
-        int rem = k;
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += kMergeThreads) hist[i] = 0;
-            __syncthreads();
-            for (int b0 = 0; b0 < total; b0 += kMergeThreads) { // warp-uniform trip count
-                const int i = b0 + tid;
-                const unsigned long long v = i < total ? mv[i] : 0ull;
-                hist_add(hist, (int)((v >> shift) & 255), i < total && (v & pmask) == prefix);
-            }
-            __syncthreads();
-            if (tid == 0) {
-                int cum = 0, b = 255;
-                for (; b > 0; --b) {
-                    if (cum + hist[b] >= rem) break;
-                    cum += hist[b];
-                }
-                s_bin = b;
-                s_rem = rem - cum;
-            }
-            __syncthreads();
-            prefix |= (unsigned long long)s_bin << shift;
-            pmask |= 255ull << shift;
-            rem = s_rem;
-            __syncthreads();
-        }
-        if (tid == 0) { s_prefix = prefix; s_cnt = 0; }
+        // the k-th largest of the unique 64-bit keys
+        unsigned long long thr64;
+        int n_gt64;
+        block_kth<kMergeThreads, unsigned long long>(total, k, [&](int i) { return mv[i]; }, &msel, thr64, n_gt64);
+        if (tid == 0) s_cnt = 0;
         __syncthreads();
-        const unsigned long long thr = s_prefix;
+        const unsigned long long thr = thr64;
         for (int i = tid; i < total; i += kMergeThreads) {
             const unsigned long long v = mv[i];
             if (v >= thr) {
@@ -485,18 +442,34 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
 
 } // namespace
 
-// Workspace bytes of the decode path (candidates + counts), and whether it serves the call.
+// Chunking of the key lists: enough chunks for about one CTA per SM, at most kChunk keys each.
+static void decode_chunks(int64_t Nq, int64_t max_nvis, int *slots, int *chunk)
+{
+    int64_t want = (148 + Nq - 1) / (Nq > 0 ? Nq : 1);
+    if (want < 1) want = 1;
+    int64_t ch = (max_nvis + want - 1) / want;
+    ch = (ch + kKT - 1) / kKT * kKT;
+    if (ch > kChunk) ch = kChunk;
+    if (ch < kKT) ch = kKT;
+    *chunk = (int)ch;
+    *slots = (int)((max_nvis + ch - 1) / ch);
+    if (*slots < 1) *slots = 1;
+}
+
+// Workspace bytes of the decode path (candidates + counts).
 size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k)
 {
-    const int64_t slots = (max_nvis + kChunk - 1) / kChunk;
-    return (size_t)Nq * (size_t)(slots > 0 ? slots : 1) * ((size_t)k * 8 + 4) + 256;
+    int slots, chunk;
+    decode_chunks(Nq, max_nvis, &slots, &chunk);
+    return (size_t)Nq * (size_t)slots * ((size_t)k * 8 + 4) + 256;
 }
 
 bool decode_indexer_eligible(const IndexerArgs &a)
 {
-    if (a.fmt != CSA_FP4 || a.H != kHI || a.d != kDI || a.Nq <= 0 || a.Nq > 65535) return false;
-    const int64_t slots = (a.max_nvis + kChunk - 1) / kChunk;
-    if (slots < 1 || slots > 64 || slots > 65535) return false;
+    if (a.fmt != CSA_FP4 || a.H != kHI || a.d != kDI || a.Nq <= 0 || a.Nq > 65535 || a.max_nvis <= 0) return false;
+    int slots, chunk;
+    decode_chunks(a.Nq, a.max_nvis, &slots, &chunk);
+    if (slots > 64) return false;
     // merge kernel: candidates (slots * k) plus the padded winner array must fit in shared memory
     int n2 = 1;
     while (n2 < a.k) n2 <<= 1;
@@ -505,13 +478,14 @@ bool decode_indexer_eligible(const IndexerArgs &a)
 
 cudaError_t launch_indexer_decode(const IndexerArgs &a, void *ws, cudaStream_t st)
 {
-    const int slots = (int)((a.max_nvis + kChunk - 1) / kChunk);
+    int slots, chunk;
+    decode_chunks(a.Nq, a.max_nvis, &slots, &chunk);
     uintptr_t p = (reinterpret_cast<uintptr_t>(ws) + 255) / 256 * 256;
     unsigned long long *cand = reinterpret_cast<unsigned long long *>(p);
     int *cnt = reinterpret_cast<int *>(cand + (size_t)a.Nq * slots * a.k);
     cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    decode_scan_kernel<<<dim3((unsigned)slots, (unsigned)a.Nq), kThreads, SMEM_ALLOC, st>>>(a, slots, cand, cnt);
+    decode_scan_kernel<<<dim3((unsigned)slots, (unsigned)a.Nq), kThreads, SMEM_ALLOC, st>>>(a, slots, chunk, cand, cnt);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int n2 = 1;

@@ -6,11 +6,12 @@
 // hold -1.
 //
 // One CTA per query row.  Radix select over order-preserving 32-bit keys of the fp32 scores
-// (four 8-bit digit passes with a shared-memory histogram) finds the exact k-th key; entries
+// (8-bit digits over the bits that differ within the row, select.cuh) finds the exact k-th key; entries
 // above it are taken unordered, entries equal to it are taken in index order by a block-wide
 // ordered scan, and the k_eff winners are then sorted in shared memory (bitonic, 64-bit keys
 // (score key, inverted index)).
 #include "common.cuh"
+#include "select.cuh"
 
 namespace csa {
 
@@ -33,9 +34,8 @@ __device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
 {
     __shared__ unsigned long long sel[TK_MAX];
-    __shared__ int hist[256];
-    __shared__ int s_bin, s_rem, s_cnt, s_warp[TK_THREADS / 32], s_eq_taken;
-    __shared__ uint32_t s_prefix;
+    __shared__ SelectSmem<uint32_t> ssel;
+    __shared__ int s_cnt, s_warp[TK_THREADS / 32], s_eq_taken;
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
@@ -47,35 +47,9 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     uint32_t thr = 0;   // k-th largest key (only meaningful when nv > k)
     int n_gt = 0;       // number of keys strictly above thr
     if (nv > k) {
-        uint32_t prefix = 0, pmask = 0;
-        int rem = k;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0;
-            __syncthreads();
-            for (int64_t b0 = 0; b0 < nv; b0 += TK_THREADS) { // warp-uniform trip count
-                const int64_t s = b0 + tid;
-                const uint32_t key = s < nv ? float_key(S[s]) : 0u;
-                hist_add(hist, (int)((key >> shift) & 255), s < nv && (key & pmask) == prefix);
-            }
-            __syncthreads();
-            if (tid == 0) {
-                int cum = 0, b = 255;
-                for (; b > 0; --b) {
-                    if (cum + hist[b] >= rem) break;
-                    cum += hist[b];
-                }
-                s_bin = b;
-                s_rem = rem - cum;
-            }
-            __syncthreads();
-            prefix |= uint32_t(s_bin) << shift;
-            pmask |= 255u << shift;
-            rem = s_rem;
-            __syncthreads();
-        }
-        thr = prefix;
-        n_gt = k - rem;
-        if (tid == 0) { s_cnt = 0; s_prefix = thr; s_eq_taken = 0; }
+        block_kth<TK_THREADS, uint32_t>((int)nv, k, [&](int i) { return float_key(S[i]); }, &ssel, thr, n_gt);
+        const int rem = k - n_gt;
+        if (tid == 0) { s_cnt = 0; s_eq_taken = 0; }
         __syncthreads();
         // strictly greater: unordered append
         for (int64_t s = tid; s < nv; s += TK_THREADS) {

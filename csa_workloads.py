@@ -92,11 +92,21 @@ def _rows(seed, name, ncols, r0, r1, draw):
     block_rows = block_rows_for(ncols)
     out = np.empty((r1 - r0, ncols), dtype=np.float32)
     b0, b1 = r0 // block_rows, (r1 - 1) // block_rows if r1 > r0 else -1
-    for b in range(b0, b1 + 1):
+
+    def fill(b):
         lo, hi = b * block_rows, (b + 1) * block_rows
         blk = draw(rng(seed, name, b), block_rows * ncols).reshape(block_rows, ncols)
         s, e = max(lo, r0), min(hi, r1)
         out[s - r0:e - r0] = blk[s - lo:e - lo]
+
+    if b1 - b0 >= 4:  # independent blocks: numpy releases the GIL while drawing
+        import concurrent.futures as cf
+        import os
+        with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(b0, b1 + 1)))
+    else:
+        for b in range(b0, b1 + 1):
+            fill(b)
     return out
 
 

@@ -76,7 +76,7 @@ typedef struct csa_kv_rows {
  * FP4 rows ([qa] Question 4, [ledger]): E2M1 elements with one E8M0 scale per 32 consecutive
  * elements (OCP MX v1.0 layout): value[j] = e2m1(nibble j) * 2^(scales[r, j/32] - 127).
  * codes [n, d/2] bytes (element 2i in the low nibble of byte i), scales [n, d/32] bytes.
- * d must be a multiple of 32; bases 16-byte aligned.
+ * d must be a multiple of 32; codes 16-byte aligned, scales 4-byte aligned.
  */
 typedef struct csa_fp4_rows {
     uint8_t *codes;

@@ -87,6 +87,7 @@ def lib():
             L.orc_dequant_fp4.argtypes = [_u8p, _u8p, _i64, _int, _f64p]
             L.orc_quant_kv.argtypes = [_f32p, _i64, _int, _int, _u8p, _u16p, _f32p]
             L.orc_dequant_kv.argtypes = [_u8p, _u16p, _f32p, _i64, _int, _int, _f64p]
+            L.orc_decode_glue.argtypes = [_f64p, _f64p, _f64p, _i64, _int, _int, _f64p, _f64p]
             L.orc_num_threads.restype = ctypes.c_int
             _lib = L
     return _lib
@@ -344,3 +345,19 @@ def dequant_kv(fp8, rope_bits, scale) -> np.ndarray:
     lib().orc_dequant_kv(_p(fp8, _u8p), _p(rope_bits, _u16p), _p(scale, _f32p), n, cn + rope, rope,
                          _p(out, _f64p))
     return out
+
+
+# ----------------------------------------------------------------------------------------
+# stacked decode workload
+# ----------------------------------------------------------------------------------------
+
+def decode_glue(o, P, Rm):
+    """Inter-layer glue of the stacked decode workload (no counterpart on the pages): returns
+    (q_next [R,c], zi [R,d]) = (RMS-normalised P o / sqrt(c), RMS-normalised Rm o), fp64."""
+    o, P, Rm = map(_f64, (o, P, Rm))
+    R, c = o.shape
+    d = Rm.shape[0]
+    qn = np.empty((R, c), np.float64)
+    zi = np.empty((R, d), np.float64)
+    lib().orc_decode_glue(_p(o, _f64p), _p(P, _f64p), _p(Rm, _f64p), R, c, d, _p(qn, _f64p), _p(zi, _f64p))
+    return qn, zi

@@ -421,3 +421,42 @@ void orc_dequant_kv(const uint8_t *fp8, const uint16_t *rope_bits, const float *
         for (int j = 0; j < rope; j++) out[r * c + cn + j] = orc_bf16_value(rope_bits[r * rope + j]);
     }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Inter-layer glue of the stacked decode workload                                             */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * The pages do not give this step: it stands in for the model's projections between the
+ * attention layers of the stacked decode workload.  For each row r of o [R, c]:
+ *   y = P o_r   (P [c, c], row-major as out x in),  q_next_r = y / rms(y) / sqrt(c)
+ *   z = Rm o_r  (Rm [d, c]),                          zi_r     = z / rms(z)
+ * with rms(v) = sqrt(mean(v^2)); a zero vector maps to zero.  q_next is the next layer's query
+ * (before bf16 storage), zi the next CSA layer's index query (before FP4 quantisation).
+ */
+void orc_decode_glue(const double *o, const double *P, const double *Rm, int64_t R, int c, int d,
+                     double *q_next, double *zi)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; r++) {
+        const double *x = o + r * c;
+        double ss = 0.0;
+        for (int i = 0; i < c; i++) {
+            double y = 0.0;
+            for (int j = 0; j < c; j++) y += P[(int64_t)i * c + j] * x[j];
+            q_next[r * c + i] = y;
+            ss += y * y;
+        }
+        double f = ss > 0.0 ? 1.0 / sqrt(ss / c) / sqrt((double)c) : 0.0;
+        for (int i = 0; i < c; i++) q_next[r * c + i] *= f;
+        ss = 0.0;
+        for (int i = 0; i < d; i++) {
+            double z = 0.0;
+            for (int j = 0; j < c; j++) z += Rm[(int64_t)i * c + j] * x[j];
+            zi[r * d + i] = z;
+            ss += z * z;
+        }
+        f = ss > 0.0 ? 1.0 / sqrt(ss / d) : 0.0;
+        for (int i = 0; i < d; i++) zi[r * d + i] *= f;
+    }
+}

@@ -342,7 +342,8 @@ def test_decode_attention_mixed_cache(C, use_idx):
                              torch.from_numpy(pos).cuda(), wkv, dev_i(win_len), dev(sink), 1.0, m, W,
                              max_nvis=int(nv.max()), idx=None if idx is None else dev_i(idx), lse=lse)
     assert row_rel_err(host(o), o_ref).max() < 2e-2
-    np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
+    # the tensor-core path rounds dequantised FP8 keys to bf16 (2^-9 relative) before the MMA
+    np.testing.assert_allclose(host(lse), lse_ref, atol=1e-2)
 
 
 # ---------------------------------------------------------------------------------------------

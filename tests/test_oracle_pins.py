@@ -448,3 +448,31 @@ def test_kv_rows_amax_maps_to_448_and_rope_is_bf16():
     z = np.zeros((2, 512), np.float32)
     f0, _, s0 = O.quant_kv(z)
     assert np.all(f0 == 0) and np.all(s0 == 1.0)
+
+
+# ---------------------------------------------------------------------------------------------
+# inter-layer glue of the stacked decode workload (not on the pages)
+# ---------------------------------------------------------------------------------------------
+
+def test_glue_normalisation_identity_and_symmetry():
+    R, c, d = 9, 16, 8
+    o = randn(R, c)
+    P, Rm = randn(c, c), randn(d, c)
+    qn, zi = O.decode_glue(o, P, Rm)
+    np.testing.assert_allclose(np.sqrt((qn ** 2).mean(1)), 1 / np.sqrt(c), rtol=1e-13)
+    np.testing.assert_allclose(np.sqrt((zi ** 2).mean(1)), 1.0, rtol=1e-13)
+    # scale invariance and odd symmetry in o
+    qn2, zi2 = O.decode_glue(3.5 * o, P, Rm)
+    np.testing.assert_allclose(qn2, qn, rtol=1e-12, atol=1e-14)
+    qn3, zi3 = O.decode_glue(-o, P, Rm)
+    np.testing.assert_allclose(qn3, -qn, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(zi3, -zi, rtol=1e-12, atol=1e-14)
+    # identity projection: the normalised input itself (the projection is P o, not P^T o)
+    qi, _ = O.decode_glue(o, np.eye(c), Rm)
+    np.testing.assert_allclose(qi, o / np.sqrt((o ** 2).mean(1, keepdims=True)) / np.sqrt(c), rtol=1e-13)
+    A = np.zeros((c, c)); A[0, 1] = 1.0; A[1, 0] = 1.0; A[2, 5] = 2.0  # non-symmetric part pins P o
+    qa, _ = O.decode_glue(o, A, Rm)
+    y = o @ A.T
+    np.testing.assert_allclose(qa, y / np.sqrt((y ** 2).mean(1, keepdims=True)) / np.sqrt(c), rtol=1e-12)
+    z0, _ = O.decode_glue(np.zeros((2, c)), P, Rm)
+    assert np.all(z0 == 0)
