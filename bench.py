@@ -7,7 +7,8 @@ tokens, bf16, c = 512 (64 RoPE dims), m' = 128 -> 256 compressed entries, 64 que
 window 128, sink.  One step = hca_compress + hybrid_attn_prefill over the whole layer.
 Other workloads (--workload): csa_prefill_64k (csa_compress x2 + indexer_topk +
 hybrid_attn_prefill), csa_decode_1m (indexer_topk FP4 + hybrid_attn_decode over the FP8/BF16
-cache, 8 sequences at position 1,048,576).
+cache, 8 sequences at position 1,048,576), mixed_decode_64 (64 sequences of log-uniform
+context length through a stack of HCA, CSA, HCA, CSA decode layers joined by csa_decode_glue).
 
 Prints ONE JSON line (rank 0).  value = tokens/s of the whole job (all ranks; each rank runs
 its own independent layer: weak scaling, no collective on the data path), measured with CUDA
@@ -330,7 +331,119 @@ class CsaDecode1M:
         self.h_out.copy_(self.o, non_blocking=True)
 
 
-WORKLOADS = {"hca_prefill_32k": HcaPrefill, "csa_prefill_64k": CsaPrefill, "csa_decode_1m": CsaDecode1M}
+class _Layer:
+    pass
+
+
+class MixedDecode:
+    """Mixed serving decode: B = 64 sequences, context lengths log-uniform in [4096, 1,048,576],
+    one new token each at t = length, through a stack of layers HCA, CSA, HCA, CSA.  Every layer
+    has its own FP8/BF16 KV cache (compressed entries + 128-row window) and sink; CSA layers add
+    FP4 index keys and index-head weights.  Layer l's output becomes layer l+1's queries (and, for
+    a CSA layer, its FP4 index queries) through csa_decode_glue.  One step = per CSA layer
+    indexer_topk + hybrid_attn_decode, per HCA layer hybrid_attn_decode, and one glue launch
+    between consecutive layers."""
+
+    def __init__(self, w, rank, torch, C, device):
+        self.w, self.torch, self.C, self.dev = w, torch, C, device
+        Bn, H, c, Hi, di, W = w.B, w.H, w.c, w.H_I, w.d_I, w.W
+        self.lens = WL.mixed_lengths(w)
+        seq0 = Bn * rank
+        self.pos = torch.from_numpy(self.lens.astype(np.int64)).to(device)
+        self.win_len = torch.full((Bn,), W, dtype=torch.int32, device=device)
+        kinds = w.extra["layers"]
+        self.layers = []
+        for l, kind in enumerate(kinds):
+            L = _Layer()
+            L.csa = kind == "csa"
+            L.m = w.extra["m_csa"] if L.csa else w.extra["m_hca"]
+            nv = (self.lens + 1) // L.m
+            L.nv, L.max_nv = nv, int(nv.max())
+            L.off_np = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+            L.off = torch.from_numpy(L.off_np).to(device)
+            n = int(nv.sum())
+            L.comp = C.KvRows.empty(n, c, w.rope, device)
+            L.keys = C.Fp4Rows.empty(n, di, device) if L.csa else None
+            chunk = 65536
+            for b in range(Bn):
+                o0 = int(L.off_np[b])
+                for r0 in range(0, int(nv[b]), chunk):
+                    r1 = min(int(nv[b]), r0 + chunk)
+                    sl = slice(o0 + r0, o0 + r1)
+                    x = torch.from_numpy(WL.draw(w, "KV", r0, r1, layer=l, seq=seq0 + b)).to(device)
+                    C.csa_quantize_kv(x, C.KvRows(L.comp.fp8[sl], L.comp.rope[sl], L.comp.scale[sl]))
+                    if L.csa:
+                        k = torch.from_numpy(WL.draw(w, "KI", r0, r1, layer=l, seq=seq0 + b)).to(device)
+                        C.csa_quantize_fp4(k, C.Fp4Rows(L.keys.codes[sl], L.keys.scales[sl]))
+            win = np.concatenate([WL.draw(w, "WIN", 0, W, layer=l, seq=seq0 + b) for b in range(Bn)])
+            L.win = C.KvRows.empty(Bn * W, c, w.rope, device)
+            C.csa_quantize_kv(torch.from_numpy(win).to(device), L.win)
+            L.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, layer=l, seq=rank)[0]).to(device)
+            L.o = torch.empty((Bn, H, c), dtype=torch.bfloat16, device=device)
+            if L.csa:
+                L.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, layer=l, seq=seq0 + b)
+                                                        for b in range(Bn)])).to(device)
+                L.qI = C.Fp4Rows.empty(Bn * Hi, di, device)
+                L.idx = torch.empty((Bn, w.k), dtype=torch.int32, device=device)
+                L.ws = torch.empty((C.indexer_topk_workspace_size(Bn, L.max_nv, w.k),), dtype=torch.uint8, device=device)
+            L.wsd = torch.empty((C.hybrid_attn_decode_workspace_size(Bn, H, c, w.k if L.csa else 0, W, L.max_nv,
+                                                                      L.csa),), dtype=torch.uint8, device=device)
+            self.layers.append(L)
+        # glue after every layer but the last: P_l, Rm_l (N(0, 1/c), bf16)
+        for l, L in enumerate(self.layers[:-1]):
+            L.P = _to_dev_bf16(WL.draw(w, "P", 0, c, layer=l), torch, device)
+            L.Rm = _to_dev_bf16(WL.draw(w, "Rm", 0, di, layer=l), torch, device) if self.layers[l + 1].csa else None
+            L.q_next = torch.empty((Bn, H, c), dtype=torch.bfloat16, device=device)
+        self.q0 = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, layer=0, seq=seq0 + b).reshape(H, c)
+                                             for b in range(Bn)])).to(torch.bfloat16).to(device)
+        if self.layers[0].csa:  # a stack that starts with CSA draws its first index query
+            qx = np.concatenate([WL.draw(w, "qI", 0, 1, layer=0, seq=seq0 + b).reshape(Hi, di) for b in range(Bn)])
+            C.csa_quantize_fp4(torch.from_numpy(qx).to(device), self.layers[0].qI)
+        torch.cuda.synchronize()
+        first = next(L for L in self.layers if L.csa)
+        self.bytes = float(first.nv.sum() * (di // 2 + di // 32))   # FP4 key scan of one CSA layer
+        self.tokens = Bn
+        self.launches_per_step = sum(4 if L.csa else 2 for L in self.layers) + len(self.layers) - 1
+        self.kernel_name = "indexer_topk (FP4 scan + top-k), first CSA layer"
+
+    def step(self, ev=None):
+        C, w = self.C, self.w
+        q = self.q0
+        timed = False
+        for l, L in enumerate(self.layers):
+            if L.csa:
+                if ev is not None and not timed:
+                    ev[0].record()
+                C.indexer_topk(L.qI, L.wI, L.keys, L.m, w.k, max_nvis=L.max_nv, q_pos=self.pos, key_off=L.off,
+                               idx_out=L.idx, workspace=L.ws)
+                if ev is not None and not timed:
+                    ev[1].record()
+                    timed = True
+            C.hybrid_attn_decode(q, L.comp, L.off, self.pos, L.win, self.win_len, L.sink, 1.0, L.m, w.W,
+                                 max_nvis=L.max_nv, idx=L.idx if L.csa else None, o=L.o, workspace=L.wsd)
+            if l + 1 < len(self.layers):
+                nxt = self.layers[l + 1]
+                C.csa_decode_glue(L.o, L.P, L.Rm, q_next=L.q_next, qI=nxt.qI if nxt.csa else None)
+                q = L.q_next
+
+    def setup_e2e(self):
+        torch = self.torch
+        self.dev_in = [self.q0, self.pos]
+        self.h_in = [t.cpu().pin_memory() for t in self.dev_in]
+        out = self.layers[-1].o
+        self.h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = out.numel() * out.element_size()
+
+    def step_e2e(self):
+        for d, h in zip(self.dev_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.layers[-1].o, non_blocking=True)
+
+
+WORKLOADS = {"hca_prefill_32k": HcaPrefill, "csa_prefill_64k": CsaPrefill, "csa_decode_1m": CsaDecode1M,
+             "mixed_decode_64": MixedDecode}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -369,6 +482,46 @@ class OracleHca:
     def describe(self):
         return (f"full hca_compress of T={self.w.T} (amortised per token) + hybrid attention of {self.n} "
                 f"query tokens evenly spaced over the layer")
+
+
+class OracleDecode:
+    """The oracle on a bounded sample of the 1M-context decode: n_seq of the batch's sequences,
+    each the full FP4 indexer scan over its 262,144 entries, the top-k, and the hybrid attention
+    over the selected FP8/BF16 rows plus the window.  Inputs are drawn and dequantised once
+    (untimed); run() times the oracle's indexer, top-k and attention."""
+
+    def __init__(self, w, n_seq: int = 1, seed_rank: int = 0):
+        import oracle as O
+        self.w, self.n = w, n_seq
+        H, c, Hi, di, W, m = w.H, w.c, w.H_I, w.d_I, w.W, w.m
+        self.t = w.T
+        self.nv = (w.T + 1) // m
+        self.seqs = []
+        for b in range(n_seq):
+            s = b + w.B * seed_rank
+            Kd = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "KI", 0, self.nv, seq=s)))
+            KV = O.dequant_kv(*O.quant_kv(WL.draw(w, "KV", 0, self.nv, seq=s)))
+            win = O.dequant_kv(*O.quant_kv(WL.draw(w, "WIN", 0, W, seq=s)))
+            q = WL.draw(w, "q", 0, 1, seq=s).reshape(1, H, c)
+            qI = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "qI", 0, 1, seq=s).reshape(Hi, di))).reshape(1, Hi, di)
+            wt = WL.draw(w, "w", 0, 1, seq=s)
+            self.seqs.append((Kd, KV, win, q, qI, wt))
+        self.sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
+
+    def run(self):
+        """Returns (tokens/s, seconds of oracle work)."""
+        import oracle as O
+        w = self.w
+        t0 = time.perf_counter()
+        for Kd, KV, win, q, qI, wt in self.seqs:
+            idx, _ = O.indexer_topk(qI, wt, Kd, np.array([self.t]), w.m, w.k)
+            O.hybrid_attn_decode(q, KV, [0], [self.t], win, [w.W], self.sink, 1.0, w.m, w.W, idx=idx)
+        secs = time.perf_counter() - t0
+        return self.n / secs, secs
+
+    def describe(self):
+        return (f"{self.n} of the {self.w.B} sequences: FP4 indexer over {self.nv} entries, top-{self.w.k}, "
+                f"hybrid attention over the selected rows + window {self.w.W}")
 
 
 def oracle_hca_sample(w, target_s: float = 10.0):
@@ -481,6 +634,16 @@ def main():
         if w.kind == "csa_decode":
             cfg.update({"B": w.B, "n_comp_per_seq": (w.T + 1) // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
                         "l2": "FP4 key scan (143 MB) and KV cache (1.2 GB) larger than L2"})
+        elif w.kind == "mixed_decode":
+            cfg = {"workload": args.workload, "B": w.B, "layers": list(w.extra["layers"]), "c": w.c,
+                   "rope_dims": w.rope, "H": w.H, "W": w.W, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+                   "m_csa": w.extra["m_csa"], "m_hca": w.extra["m_hca"],
+                   "context": f"log-uniform [{w.extra['len_lo']}, {w.extra['len_hi']}]",
+                   "total_context_tokens": int(job.lens.sum()), "parallelism": f"replicas x{world}",
+                   "l2": "KV caches of the stack ({:.2f} GB) larger than L2".format(
+                       sum(L.comp.fp8.numel() + L.comp.rope.numel() * 2 + L.comp.scale.numel() * 4
+                           + (L.keys.codes.numel() + L.keys.scales.numel() if L.csa else 0)
+                           for L in job.layers) / 1e9)}
         elif w.kind == "csa_prefill":
             cfg.update({"n_comp": w.T // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
                         "l2": "inputs larger than L2 (q alone is 4.3 GB)"})
@@ -506,9 +669,14 @@ def main():
             "clocks": clk.summary(),
             "gpu_launches": job.launches_per_step * args.steps,
         }
-        if not args.no_cpu_baseline and world == 1 and args.workload == "hca_prefill_32k":
+        if not args.no_cpu_baseline and world == 1 and args.workload in ("hca_prefill_32k", "csa_decode_1m"):
             import oracle as O
-            tps, secs, desc = oracle_hca_sample(w)
+            if args.workload == "hca_prefill_32k":
+                tps, secs, desc = oracle_hca_sample(w)
+            else:
+                job_o = OracleDecode(w, 4)
+                tps, secs = job_o.run()
+                desc = job_o.describe()
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
                                     "sample": desc, "seconds": secs}
         print(json.dumps(line), flush=True)
@@ -522,13 +690,13 @@ def reference_arm(args, w, world, rank):
     if rank != 0:
         return
     import oracle as O
-    job = OracleHca(w, 256)
+    job = OracleDecode(w, 1) if w.kind == "csa_decode" else OracleHca(w, 256)
     desc = job.describe()
     for _ in range(max(args.warmup, 3)):
         job.run()
     vals, secs = [], []
     for _ in range(args.steps):
-        tps, s, _, _ = job.run()
+        tps, s = job.run()[:2]
         vals.append(tps)
         secs.append(s)
     value = statistics.median(vals)

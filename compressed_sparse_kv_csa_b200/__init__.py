@@ -24,6 +24,7 @@ CSA_ERR_CUDA = -3
 CSA_ERR_WORKSPACE = -5
 CSA_DEVERR_TIMEOUT = 1
 CSA_DEVERR_INDEX = 2
+CSA_DEVERR_RANGE = 4
 CSA_F32 = 0
 CSA_BF16 = 1
 CSA_FP4 = 2
@@ -73,6 +74,7 @@ def _load():
         "indexer_topk_static_capacity": ([], sz),
         "indexer_topk_static": ([vp, vp, vp, i32, vp, vp, i64, i64, i32, i32, i32, i32, i64, vp, vp, vp],
                                 ctypes.c_int),
+        "csa_decode_glue": ([vp, vp, vp, i64, i32, i32, vp, P_f4, vp], ctypes.c_int),
         "csa_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
         "csa_status_string": ([i32], ctypes.c_char_p),
         "csa_abi_version": ([], i32),
@@ -311,6 +313,23 @@ def hybrid_attn_decode(q, comp: KvRows, comp_off, pos, win: KvRows, win_len, sin
                                  _stream(stream))
     _check("hybrid_attn_decode", st)
     return o
+
+
+def csa_decode_glue(o, P, Rm=None, q_next=None, qI: Fp4Rows | None = None, stream=None):
+    """Inter-layer projection of a decode stack: q_next = bf16(RMS-normalised P o / sqrt(c)) and,
+    when Rm is given, qI = FP4(RMS-normalised Rm o).  o is [..., c] bf16 (rows = sequences x
+    heads); returns (q_next shaped like o, qI or None)."""
+    c = o.shape[-1]
+    R = o.numel() // c if c else 0
+    if q_next is None:
+        q_next = torch.empty_like(o)
+    d = Rm.shape[0] if Rm is not None else 0
+    if Rm is not None and qI is None:
+        qI = Fp4Rows.empty(R, d, o.device)
+    st = _lib.csa_decode_glue(_ptr(o), _ptr(P), _ptr(Rm), R, c, d, _ptr(q_next),
+                              ctypes.byref(qI._c()) if qI is not None else None, _stream(stream))
+    _check("csa_decode_glue", st)
+    return q_next, qI
 
 
 def csa_device_error(stream=None) -> int:

@@ -31,6 +31,8 @@ int decode_tc_chunks(int64_t max_keys);
 bool decode_attn_tc_eligible(const DecodeArgs &a);
 cudaError_t launch_attn_decode_tc(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int c, int d,
+                               void *q_next, const Fp4RowsDev *qI, int *err, cudaStream_t st);
 } // namespace csa
 
 using namespace csa;
@@ -305,6 +307,25 @@ int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *co
     }
     decode_plan(B, H, c, (int)max_keys, &a.n_chunks, &a.chunk);
     return status_of(launch_attn_decode(a, S(stream)));
+}
+
+// ------------------------------------------------------------------------------------------
+
+int csa_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int32_t c, int32_t d,
+                    void *q_next, const csa_fp4_rows *qI, void *stream)
+{
+    if (!o || !P || !q_next || R < 0 || R >= (1ll << 31)) return CSA_ERR_INVALID_ARG;
+    if (c < 64 || c > 512 || c % 64) return CSA_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(P) || !aligned16(q_next)) return CSA_ERR_INVALID_ARG;
+    if (qI) {
+        if (!Rm || !aligned16(Rm) || d < 32 || d > 256 || d % 32 || !fp4_rows_ok(qI, R, d)) return CSA_ERR_INVALID_ARG;
+    }
+    if (R == 0) return CSA_OK;
+    Fp4RowsDev q4{};
+    if (qI) q4 = to_dev(*qI);
+    const cudaError_t e = launch_decode_glue(o, P, Rm, R, c, d, q_next, qI ? &q4 : nullptr, dev_error_word(), S(stream));
+    if (e == cudaErrorInvalidValue) return CSA_ERR_INVALID_ARG;
+    return status_of(e);
 }
 
 } // extern "C"

@@ -12,7 +12,8 @@
 //     into a 4-stage ring;
 //   * 8 converter warps turn a tile into f16 in the 128-byte-swizzled MMA layout with the
 //     hardware E2M1x2 -> f16x2 conversion, folding each block's power-of-two scale in with one
-//     f16x2 multiply (exact while the block's scale exponent lies in [-23, 13]);
+//     f16x2 multiply (exact while the block's scale exponent lies in [-23, 13]; a non-zero block
+//     outside that range sets CSA_DEVERR_RANGE, its scores are then approximate);
 //   * one lane issues tcgen05 M=128 (keys) x N=64 (heads) x K=128 f16 MMAs against the query,
 //     converted the same way once per CTA, into a double-buffered TMEM accumulator;
 //   * 4 epilogue warps (one per TMEM lane quadrant) reduce w . ReLU(.) over the 64 heads per key
@@ -76,6 +77,15 @@ __device__ __forceinline__ uint32_t f16_pow2x2(int e)
     if (e >= -14) b = (uint32_t)((e > 15 ? 15 : e) + 15) << 10;
     else b = (e >= -24) ? (1u << (e + 24)) : 0u;
     return b | (b << 16);
+}
+
+// E2M1 magnitudes are m * 2^e with m in [0.5, 6]: in f16 exactly for block exponents e in
+// [-23, 13] (the smallest, 0.5 * 2^-23, is f16's smallest subnormal; the largest, 6 * 2^13,
+// is below 65504).  An all-zero block is exact for any scale.
+__device__ __forceinline__ bool fp4_block_exact_f16(uint32_t scale_byte, uint4 codes)
+{
+    const bool zero = ((codes.x | codes.y | codes.z | codes.w) & 0x77777777u) == 0u;
+    return zero || (scale_byte >= 127u - 23u && scale_byte <= 127u + 13u);
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t x, uint32_t y)
@@ -238,9 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
         const int h = tid >> 2, blk = tid & 3;
         const int64_t qr = r * kHI + h;
         const uint4 codes = *reinterpret_cast<const uint4 *>(a.q4.codes + qr * (kDI / 2) + 16 * blk);
-        const int e = (int)a.q4.scales[qr * (kDI / 32) + blk] - 127;
+        const uint32_t sb = a.q4.scales[qr * (kDI / 32) + blk];
         uint32_t v[16];
-        e2m1x32_to_f16(codes, e, v);
+        e2m1x32_to_f16(codes, (int)sb - 127, v);
+        if (!fp4_block_exact_f16(sb, codes)) flag_error(a.err, CSA_DEVERR_RANGE);
         store_block(base + OFF_B, 8192u, h, blk, v);
     } else if (tid < 256 + 64) {
         const int h = tid - 256;
@@ -276,6 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
         }
     } else if (warp >= kConvWarp0 && warp < kEpiWarp0) {
         const int ct = tid - 32 * kConvWarp0; // 0 .. 32*kConvWarps-1
+        bool out_of_range = false;            // a non-zero block whose scale f16 cannot carry exactly
         for (int i = 0; i < ntiles && ok; ++i) {
             const uint32_t st = i % kStages, ab = i & 1;
             if (!wwait(bar(B_STFULL + st), (i / kStages) & 1)) { ok = false; break; }
@@ -294,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
                     uint32_t sb;
                     asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sb) : "r"(stb + kStageCodes + (uint32_t)key * 4u + blk));
                     e2m1x32_to_f16(codes, (int)sb - 127, v);
+                    out_of_range |= !fp4_block_exact_f16(sb, codes);
                 } else {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0u;
@@ -304,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             mbar_arrive(bar(B_STEMPTY + st));
             mbar_arrive(bar(B_AFULL + ab));
         }
+        if (out_of_range) flag_error(a.err, CSA_DEVERR_RANGE);
     } else if (warp >= kEpiWarp0 && warp < kMmaWarp) {
         const int quad = warp & 3;
         const float *wsm = reinterpret_cast<const float *>(sp + OFF_W);
@@ -442,10 +456,11 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
 
 } // namespace
 
-// Chunking of the key lists: enough chunks for about one CTA per SM, at most kChunk keys each.
+// Chunking of the key lists: at most one CTA per SM of the B200's 148 (the CTAs of one launch fill
+// a single wave: a 149th CTA would double the launch time), at most kChunk keys each.
 static void decode_chunks(int64_t Nq, int64_t max_nvis, int *slots, int *chunk)
 {
-    int64_t want = (148 + Nq - 1) / (Nq > 0 ? Nq : 1);
+    int64_t want = 148 / (Nq > 0 ? Nq : 1);
     if (want < 1) want = 1;
     int64_t ch = (max_nvis + want - 1) / want;
     ch = (ch + kKT - 1) / kKT * kKT;

@@ -157,6 +157,9 @@ def draw(w: Workload, name: str, r0: int = 0, r1: int | None = None, layer: int 
       sink [1,H]             sink logits, N(0,1), fp32
       KV [N,c]               compressed KV entries before quantisation (decode), N(0,1)
       WIN [W,c]              window KV rows before quantisation (decode), N(0,1)
+      P [c,c]                inter-layer query projection of the stacked decode (row i = output
+                             channel i), N(0, 1/c)
+      Rm [d_I,c]             inter-layer index-query projection of the stacked decode, N(0, 1/c)
     """
     tag = f"{name}/L{layer}/S{seq}"
     std = 1.0
@@ -165,12 +168,12 @@ def draw(w: Workload, name: str, r0: int = 0, r1: int | None = None, layer: int 
         "Ca": w.c, "Cb": w.c, "Za": w.c, "Zb": w.c, "C": w.c, "Z": w.c,
         "B": w.c, "CIa": w.d_I, "CIb": w.d_I, "ZIa": w.d_I, "ZIb": w.d_I, "BI": w.d_I,
         "KI": w.d_I, "qI": w.H_I * w.d_I, "w": w.H_I, "X": w.c, "q": w.H * w.c,
-        "sink": w.H, "KV": w.c, "WIN": w.c,
+        "sink": w.H, "KV": w.c, "WIN": w.c, "P": w.c, "Rm": w.c,
     }
     ncols = dims[name]
     if name in ("B", "BI"):
         std = w.bias_std
-    if name == "q":
+    if name in ("q", "P", "Rm"):
         std = 1.0 / np.sqrt(w.c)
     if r1 is None:
         r1 = {"sink": 1}.get(name, r0 + 1)

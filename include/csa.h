@@ -49,6 +49,8 @@ extern "C" {
 /* device error word bits (csa_device_error) */
 #define CSA_DEVERR_TIMEOUT 1       /* a bounded wait ran out */
 #define CSA_DEVERR_INDEX 2         /* an out-of-range index was skipped */
+#define CSA_DEVERR_RANGE 4         /* FP4 decode indexer: a non-zero block scale outside 2^-23..2^13
+                                      met the exact-f16 tensor-core path; those scores are inexact */
 
 #define CSA_F32 0
 #define CSA_BF16 1
@@ -234,6 +236,26 @@ int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *co
                        const int32_t *idx, int32_t k, const float *sink, float scale, int32_t B,
                        int32_t H, int32_t c, int32_t m, int32_t W, int64_t max_nvis, void *o,
                        float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * csa_decode_glue -- inter-layer projection for a stack of decode layers.  The pages describe a
+ * single attention layer and give no counterpart: this is a fixed random projection that turns
+ * one layer's attention output into the next layer's queries, so that several layers can run
+ * back to back on a decode batch.  Per row r (one row per sequence and head):
+ *     y = P o[r],   q_next[r] = bf16( y / rms(y) / sqrt(c) )
+ *     z = Rm o[r],  qI rows r = FP4( z / rms(z) )      (index query of a following CSA layer)
+ * with rms(v) = sqrt(mean(v^2)); an all-zero y or z gives an all-zero output row.  The FP4 rows
+ * use the index-key format of csa_quantize_fp4 (same scale rule, round to nearest even).
+ *   o       [R, c] bf16 (R = sequences x heads), 16-byte aligned
+ *   P       [c, c] bf16, row i = output channel i (y_i = sum_j P[i,j] o_j), 16-byte aligned
+ *   Rm      [d, c] bf16 or NULL when qI is NULL, 16-byte aligned
+ *   q_next  [R, c] bf16 out, 16-byte aligned
+ *   qI      FP4 rows out (->n >= R, ->d == d) or NULL (next layer has no indexer)
+ * fp32 accumulation on the tensor cores.  Limits: c a multiple of 64 in [64, 512]; d a multiple
+ * of 32 in [32, 256]; R < 2^31.  Caller-owned memory, nothing allocated; -1 on bad arguments.
+ */
+int csa_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int32_t c, int32_t d,
+                    void *q_next, const csa_fp4_rows *qI, void *stream);
 
 /* ----------------------------------------------------------------------------------------- */
 

@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
 CPU-baseline leg may import this package.  The product path (``compressed_sparse_kv_csa_b200``)
 never imports it, and this package never imports the product: the two share no code.  The only
-shared module is the seeded input generator (``compressed_sparse_kv_csa_b200.workloads``), which
+shared module is the seeded input generator (``csa_workloads``, at the repository root), which
 holds no arithmetic of the method.
 
 The arithmetic lives in ``csa_oracle.c`` (plain fp64 C loops, OpenMP over rows).  This module

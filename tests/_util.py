@@ -45,3 +45,30 @@ def check_topk(idx_gpu: np.ndarray, idx_orc: np.ndarray, S_orc: np.ndarray, nvis
         for s in set(gs.tolist()) ^ set(o.tolist()):
             assert abs(S_orc[r, s] - kth) <= tol, (r, s, S_orc[r, s], kth)
     return same
+
+
+def check_fp4_near(codes_g, scales_g, x, atol: float = 2e-5, max_frac: float = 1e-3):
+    """FP4 rows (E2M1 codes, E8M0 scale per 32) quantised on the GPU from values that the GPU
+    computed itself, against the oracle's fp64 values x [n, d] of the same quantity.  The
+    quantiser's decisions agree with the oracle's quantisation of x except where x lies within
+    atol of a decision boundary (the GPU's pre-quantisation value differs from x by its fp32
+    accumulation error): a different block scale needs the block amax within atol of 6*2^e, a
+    different code needs the GPU's value to be as near to x as the oracle's, up to 2*atol.
+    Returns the number of elements that differ from the oracle's quantisation."""
+    import oracle as O
+    x = np.asarray(x, np.float64)
+    n, d = x.shape
+    codes_r, scales_r = O.quant_fp4(x.astype(np.float32))
+    ds = scales_g.astype(np.int64) != scales_r.astype(np.int64)
+    if ds.any():
+        amax = np.abs(x.reshape(n, d // 32, 32)).max(-1)
+        e = np.minimum(scales_g.astype(np.int64), scales_r.astype(np.int64)) - 127
+        bound = 6.0 * np.ldexp(1.0, e)
+        assert np.all(np.abs(amax - bound)[ds] <= atol), "block scale differs away from a boundary"
+    vg, vr = O.dequant_fp4(codes_g, scales_g), O.dequant_fp4(codes_r, scales_r)
+    diff = vg != vr
+    blk_same = np.repeat(~ds, 32, axis=1)
+    bad = diff & blk_same & (np.abs(vg - x) > np.abs(vr - x) + 2 * atol)
+    assert not bad.any(), ("FP4 code differs away from a rounding boundary", np.argwhere(bad)[:4])
+    assert diff.mean() <= max_frac, diff.mean()
+    return int(diff.sum())

@@ -102,3 +102,18 @@ def test_indexer_and_attention_reject_bad_arguments(C):
 
 def test_device_error_rejects_null(C):
     assert C.lib().csa_device_error(None, None) == C.CSA_ERR_INVALID_ARG
+
+
+def test_decode_glue_rejects_bad_arguments(C):
+    L = C.lib()
+    f = FAKE
+    f4 = C._Fp4Rows(0x100000, 0x200000, 256, 128)
+    ok = lambda: ctypes.byref(f4)
+    assert L.csa_decode_glue(None, f, f, 256, 512, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG
+    assert L.csa_decode_glue(f, f, f, 256, 96, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG     # c % 64
+    assert L.csa_decode_glue(f, f, f, 256, 576, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG    # c > 512
+    assert L.csa_decode_glue(f, f, f, 256, 512, 48, f, ok(), None) == C.CSA_ERR_INVALID_ARG     # d % 32
+    assert L.csa_decode_glue(f, f, None, 256, 512, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG  # qI without Rm
+    assert L.csa_decode_glue(f, f, f, 257, 512, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG    # qI too short
+    assert L.csa_decode_glue(f, MISALIGNED, f, 256, 512, 128, f, ok(), None) == C.CSA_ERR_INVALID_ARG
+    assert L.csa_decode_glue(f, f, None, 0, 512, 0, f, None, None) == C.CSA_OK                 # nothing to do

@@ -13,7 +13,7 @@ import torch
 
 import csa_workloads as WL
 import oracle as O
-from _util import check_topk, dev, host, row_rel_err
+from _util import check_fp4_near, check_topk, dev, host, row_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -376,3 +376,37 @@ def test_tiny_csa_layer_end_to_end(C):
     assert same.sum() >= T - 8
     err = row_rel_err(host(o)[same], o_ref[same])
     assert err.max() < 1e-4, err.max()
+
+
+# ---------------------------------------------------------------------------------------------
+# inter-layer glue of the stacked decode workload
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("R,c,d", [(4096, 512, 128), (300, 512, 128), (130, 256, 64), (64, 128, 32), (1, 64, 32)])
+def test_decode_glue(C, R, c, d):
+    """q_next = bf16(RMS-normalised P o / sqrt(c)) and qI = FP4(RMS-normalised Rm o) against the
+    oracle's fp64 glue.  bf16 rounding bounds q_next at 2^-8 relative per element (5e-3 with the
+    fp32 accumulation); the FP4 codes agree except where a value sits on a rounding boundary.
+    Rows 0 and R-1 are all-zero inputs, which map to zero outputs."""
+    seed = WL.SEED_BASE + 5
+    o = WL.on_grid(WL.normal_rows(seed, f"glue_o/{R}", c, 0, R), "bf16")
+    o[0] = 0.0
+    o[R - 1] = 0.0
+    P = WL.on_grid(WL.normal_rows(seed, f"glue_P/{c}", c, 0, c, std=1 / np.sqrt(c)), "bf16")
+    Rm = WL.on_grid(WL.normal_rows(seed, f"glue_R/{c}/{d}", c, 0, d, std=1 / np.sqrt(c)), "bf16")
+    qn, zi = O.decode_glue(o, P, Rm)
+    q_g, qI = C.csa_decode_glue(dev(o, "bf16"), dev(P, "bf16"), dev(Rm, "bf16"))
+    torch.cuda.synchronize()
+    assert C.csa_device_error() == 0
+    qg = host(q_g)
+    live = np.abs(qn).max(-1) > 0
+    assert np.all(qg[~live] == 0)
+    if live.any():
+        assert row_rel_err(qg[live], qn[live]).max() <= 5e-3
+    codes, scales = qI.codes.cpu().numpy(), qI.scales.cpu().numpy()
+    assert np.all(codes[~live] == 0) and np.all(scales[~live] == 0)
+    check_fp4_near(codes, scales, zi)
+    # without an index query only q_next is written
+    q2, none = C.csa_decode_glue(dev(o, "bf16"), dev(P, "bf16"))
+    assert none is None
+    assert torch.equal(q2, q_g)
