@@ -49,6 +49,24 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def max_over_ranks(values, world: int, dist, device):
+    """Element-wise max of the per-rank values over all ranks (the job's time is its slowest
+    rank's); identity on one rank."""
+    values = [float(v) for v in values]
+    if world == 1:
+        return values
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def rank_sequences(n_seq: int, rank: int):
+    """Seed indices of the sequences a rank draws: every rank gets its own n_seq sequences (weak
+    scaling, no data shared between ranks)."""
+    return [rank * n_seq + b for b in range(n_seq)]
+
+
 # ---------------------------------------------------------------------------------------------
 # algorithmic work
 # ---------------------------------------------------------------------------------------------
@@ -264,6 +282,7 @@ class CsaDecode1M:
     def __init__(self, w, rank, torch, C, device):
         self.w, self.torch, self.C, self.dev = w, torch, C, device
         Bn, H, c, Hi, di, W, m = w.B, w.H, w.c, w.H_I, w.d_I, w.W, w.m
+        seqs = rank_sequences(Bn, rank)
         t = w.T
         nv = (t + 1) // m
         self.nv = nv
@@ -273,22 +292,22 @@ class CsaDecode1M:
         for b in range(Bn):
             for r0 in range(0, nv, chunk):
                 r1 = min(nv, r0 + chunk)
-                x = torch.from_numpy(WL.draw(w, "KV", r0, r1, seq=b + 8 * rank)).to(device)
+                x = torch.from_numpy(WL.draw(w, "KV", r0, r1, seq=seqs[b])).to(device)
                 C.csa_quantize_kv(x, C.KvRows(self.comp.fp8[b * nv + r0:b * nv + r1], self.comp.rope[b * nv + r0:b * nv + r1],
                                               self.comp.scale[b * nv + r0:b * nv + r1]))
-                k = torch.from_numpy(WL.draw(w, "KI", r0, r1, seq=b + 8 * rank)).to(device)
+                k = torch.from_numpy(WL.draw(w, "KI", r0, r1, seq=seqs[b])).to(device)
                 C.csa_quantize_fp4(k, C.Fp4Rows(self.keys.codes[b * nv + r0:b * nv + r1],
                                                 self.keys.scales[b * nv + r0:b * nv + r1]))
-        win = torch.from_numpy(np.concatenate([WL.draw(w, "WIN", 0, W, seq=b + 8 * rank) for b in range(Bn)])).to(device)
+        win = torch.from_numpy(np.concatenate([WL.draw(w, "WIN", 0, W, seq=seqs[b]) for b in range(Bn)])).to(device)
         self.win = C.KvRows.empty(Bn * W, c, w.rope, device)
         C.csa_quantize_kv(win, self.win)
-        self.q = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, seq=b + 8 * rank).reshape(H, c)
+        self.q = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, seq=seqs[b]).reshape(H, c)
                                             for b in range(Bn)])).to(torch.bfloat16).to(device)
-        qx = torch.from_numpy(np.concatenate([WL.draw(w, "qI", 0, 1, seq=b + 8 * rank).reshape(Hi, di)
+        qx = torch.from_numpy(np.concatenate([WL.draw(w, "qI", 0, 1, seq=seqs[b]).reshape(Hi, di)
                                               for b in range(Bn)])).to(device)
         self.qI = C.Fp4Rows.empty(Bn * Hi, di, device)
         C.csa_quantize_fp4(qx, self.qI)
-        self.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, seq=b + 8 * rank) for b in range(Bn)])).to(device)
+        self.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, seq=seqs[b]) for b in range(Bn)])).to(device)
         self.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, seq=rank)[0]).to(device)
         self.pos = torch.full((Bn,), t, dtype=torch.int64, device=device)
         self.key_off = torch.arange(Bn, dtype=torch.int64, device=device) * nv
@@ -348,7 +367,7 @@ class MixedDecode:
         self.w, self.torch, self.C, self.dev = w, torch, C, device
         Bn, H, c, Hi, di, W = w.B, w.H, w.c, w.H_I, w.d_I, w.W
         self.lens = WL.mixed_lengths(w)
-        seq0 = Bn * rank
+        seqs = rank_sequences(Bn, rank)
         self.pos = torch.from_numpy(self.lens.astype(np.int64)).to(device)
         self.win_len = torch.full((Bn,), W, dtype=torch.int32, device=device)
         kinds = w.extra["layers"]
@@ -370,18 +389,18 @@ class MixedDecode:
                 for r0 in range(0, int(nv[b]), chunk):
                     r1 = min(int(nv[b]), r0 + chunk)
                     sl = slice(o0 + r0, o0 + r1)
-                    x = torch.from_numpy(WL.draw(w, "KV", r0, r1, layer=l, seq=seq0 + b)).to(device)
+                    x = torch.from_numpy(WL.draw(w, "KV", r0, r1, layer=l, seq=seqs[b])).to(device)
                     C.csa_quantize_kv(x, C.KvRows(L.comp.fp8[sl], L.comp.rope[sl], L.comp.scale[sl]))
                     if L.csa:
-                        k = torch.from_numpy(WL.draw(w, "KI", r0, r1, layer=l, seq=seq0 + b)).to(device)
+                        k = torch.from_numpy(WL.draw(w, "KI", r0, r1, layer=l, seq=seqs[b])).to(device)
                         C.csa_quantize_fp4(k, C.Fp4Rows(L.keys.codes[sl], L.keys.scales[sl]))
-            win = np.concatenate([WL.draw(w, "WIN", 0, W, layer=l, seq=seq0 + b) for b in range(Bn)])
+            win = np.concatenate([WL.draw(w, "WIN", 0, W, layer=l, seq=seqs[b]) for b in range(Bn)])
             L.win = C.KvRows.empty(Bn * W, c, w.rope, device)
             C.csa_quantize_kv(torch.from_numpy(win).to(device), L.win)
             L.sink = torch.from_numpy(WL.draw(w, "sink", 0, 1, layer=l, seq=rank)[0]).to(device)
             L.o = torch.empty((Bn, H, c), dtype=torch.bfloat16, device=device)
             if L.csa:
-                L.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, layer=l, seq=seq0 + b)
+                L.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, 1, layer=l, seq=seqs[b])
                                                         for b in range(Bn)])).to(device)
                 L.qI = C.Fp4Rows.empty(Bn * Hi, di, device)
                 L.idx = torch.empty((Bn, w.k), dtype=torch.int32, device=device)
@@ -394,10 +413,10 @@ class MixedDecode:
             L.P = _to_dev_bf16(WL.draw(w, "P", 0, c, layer=l), torch, device)
             L.Rm = _to_dev_bf16(WL.draw(w, "Rm", 0, di, layer=l), torch, device) if self.layers[l + 1].csa else None
             L.q_next = torch.empty((Bn, H, c), dtype=torch.bfloat16, device=device)
-        self.q0 = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, layer=0, seq=seq0 + b).reshape(H, c)
+        self.q0 = torch.from_numpy(np.stack([WL.draw(w, "q", 0, 1, layer=0, seq=seqs[b]).reshape(H, c)
                                              for b in range(Bn)])).to(torch.bfloat16).to(device)
         if self.layers[0].csa:  # a stack that starts with CSA draws its first index query
-            qx = np.concatenate([WL.draw(w, "qI", 0, 1, layer=0, seq=seq0 + b).reshape(Hi, di) for b in range(Bn)])
+            qx = np.concatenate([WL.draw(w, "qI", 0, 1, layer=0, seq=seqs[b]).reshape(Hi, di) for b in range(Bn)])
             C.csa_quantize_fp4(torch.from_numpy(qx).to(device), self.layers[0].qI)
         torch.cuda.synchronize()
         first = next(L for L in self.layers if L.csa)
@@ -592,10 +611,7 @@ def main():
         dist.barrier()
     ms = start.elapsed_time(stop) / args.steps
     kern_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    t = torch.tensor([ms, kern_ms], device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, kern_ms = float(t[0]), float(t[1])
+    ms, kern_ms = max_over_ranks([ms, kern_ms], world, dist, device)
 
     # end to end through the C ABI with host buffers
     job.setup_e2e()
@@ -610,11 +626,9 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    te = torch.tensor([e2e_ms], device=device)
+    (e2e_ms,) = max_over_ranks([e2e_ms], world, dist, device)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(te[0])
 
     if rank == 0:
         pk, src = peaks()

@@ -24,7 +24,6 @@ CSA_ERR_CUDA = -3
 CSA_ERR_WORKSPACE = -5
 CSA_DEVERR_TIMEOUT = 1
 CSA_DEVERR_INDEX = 2
-CSA_DEVERR_RANGE = 4
 CSA_F32 = 0
 CSA_BF16 = 1
 CSA_FP4 = 2

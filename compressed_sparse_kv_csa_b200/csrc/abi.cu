@@ -49,7 +49,7 @@ bool kv_rows_ok(const csa_kv_rows *kv, int64_t n_min, int32_t c)
     if (!kv || !kv->fp8 || !kv->scale || kv->c != c || kv->n < n_min) return false;
     if (kv->rope_dims < 0 || kv->rope_dims > c || (kv->rope_dims % 16) || ((c - kv->rope_dims) % 16)) return false;
     if (kv->rope_dims > 0 && (!kv->rope || !aligned16(kv->rope))) return false;
-    return aligned16(kv->fp8) && aligned16(kv->scale);
+    return aligned16(kv->fp8) && (reinterpret_cast<uintptr_t>(kv->scale) & 3u) == 0;
 }
 
 bool fp4_rows_ok(const csa_fp4_rows *f, int64_t n_min, int32_t d)

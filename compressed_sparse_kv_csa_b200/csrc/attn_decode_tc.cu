@@ -32,7 +32,8 @@ constexpr uint32_t OFF_Q = 0;        // 8 sub-tiles [64 x 128 B]   64 KB
 constexpr uint32_t OFF_K = 65536;    // 8 sub-tiles [128 x 128 B]  128 KB
 constexpr uint32_t OFF_P = 196608;   // 2 sub-tiles [64 x 128 B]   16 KB
 constexpr uint32_t OFF_VALID = 212992; // 128 flags
-constexpr uint32_t OFF_BAR = OFF_VALID + 512;
+constexpr uint32_t OFF_ROWS = OFF_VALID + 512; // 128 resolved key rows (int64)
+constexpr uint32_t OFF_BAR = OFF_ROWS + 1024;
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = OFF_TMEM + 64 + 1024;
 constexpr uint32_t TMEM_O = 16u << 16;
@@ -114,41 +115,85 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
     }
     if (warp == kMmaWarp) tmem_alloc(base + OFF_TMEM, 512);
 
-    // ---- stage q and gather the chunk's key rows (all 288 threads)
-    for (int e = tid; e < kH * (kC / 8); e += kThreads) {
-        const int h = e >> 6, cc = e & 63;
-        const uint4 v = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + h) * kC + 8 * cc);
-        sts4(sQ + (uint32_t)(cc >> 3) * 8192u + sw128_off(h, (cc & 7) * 8), v);
-    }
-    const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
-    for (int e = tid; e < kKT * (kC / 8); e += kThreads) {
-        const int jj = e >> 6, cc = e & 63; // key slot, 8-channel chunk
-        const int64_t j = j0 + jj;
-        const KvRowsDev *kv = nullptr;
-        int64_t row = -1;
+    // ---- resolve the chunk's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
+    int64_t *rows = reinterpret_cast<int64_t *>(sp + OFF_ROWS);
+    if (tid < kKT) {
+        const int64_t j = j0 + tid;
+        int64_t code = -1;
         if (j < n_keys && j < n_win) {
-            kv = &a.win;
-            row = (int64_t)b * a.W + j;
+            code = (int64_t)b * a.W + j;
         } else if (j < n_keys) {
             const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
             if (s >= 0) {
                 const int64_t r = a.comp_off[b] + s;
-                if (r >= 0 && r < a.comp.n) {
-                    kv = &a.comp;
-                    row = r;
-                } else if (cc == 0) {
-                    flag_error(a.err, CSA_DEVERR_INDEX);
+                if (r >= 0 && r < a.comp.n) code = r | (1ll << 62);
+                else flag_error(a.err, CSA_DEVERR_INDEX);
+            }
+        }
+        rows[tid] = code;
+        valid[tid] = code >= 0 ? 1 : 0;
+    }
+    // ---- stage q (all threads): 16 independent 16-byte loads per thread in flight
+    for (int e0 = tid; e0 < kH * (kC / 8); e0 += 16 * kThreads) {
+        uint4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int e = e0 + u * kThreads;
+            if (e < kH * (kC / 8))
+                v[u] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + (e >> 6)) * kC + 8 * (e & 63)));
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int e = e0 + u * kThreads;
+            if (e < kH * (kC / 8)) {
+                const int h = e >> 6, cc = e & 63;
+                sts4(sQ + (uint32_t)(cc >> 3) * 8192u + sw128_off(h, (cc & 7) * 8), v[u]);
+            }
+        }
+    }
+    __syncthreads();
+    // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as is;
+    // 12 independent loads per thread in flight
+    const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
+    constexpr int kU = 12;
+    for (int e0 = tid; e0 < kKT * (kC / 8); e0 += kU * kThreads) {
+        uint4 raw[kU];
+        float sc[kU];
+        int kind[kU]; // 0 empty, 1 FP8, 2 RoPE
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * kThreads;
+            kind[u] = 0;
+            raw[u] = make_uint4(0, 0, 0, 0);
+            sc[u] = 0.f;
+            if (e < kKT * (kC / 8)) {
+                const int64_t code = rows[e >> 6];
+                if (code >= 0) {
+                    const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
+                    const int64_t row = code & ((1ll << 62) - 1);
+                    const int ch = 8 * (e & 63);
+                    if (ch < cn) {
+                        const uint2 c = __ldg(reinterpret_cast<const uint2 *>(kv.fp8 + row * cn + ch));
+                        raw[u].x = c.x;
+                        raw[u].y = c.y;
+                        sc[u] = __ldg(kv.scale + row);
+                        kind[u] = 1;
+                    } else {
+                        raw[u] = __ldg(reinterpret_cast<const uint4 *>(kv.rope + row * kv.rope_dims + (ch - cn)));
+                        kind[u] = 2;
+                    }
                 }
             }
         }
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (kv) {
-            const int ch = 8 * cc;
-            if (ch < cn) v = fp8x8_to_bf16(*reinterpret_cast<const uint2 *>(kv->fp8 + row * cn + ch), kv->scale[row]);
-            else v = *reinterpret_cast<const uint4 *>(kv->rope + row * kv->rope_dims + (ch - cn));
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * kThreads;
+            if (e < kKT * (kC / 8)) {
+                const int jj = e >> 6, cc = e & 63;
+                const uint4 v = kind[u] == 1 ? fp8x8_to_bf16(make_uint2(raw[u].x, raw[u].y), sc[u]) : raw[u];
+                sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
+            }
         }
-        sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
-        if (cc == 0) valid[jj] = kv ? 1 : 0;
     }
     fence_proxy_async_smem();
     tc_fence_before();

@@ -270,41 +270,61 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
 // The per-chunk weights e^{m_j - m} / denominator are computed once into shared memory.
 constexpr int kMaxMergeChunks = 1024;
 
-__global__ void decode_merge_kernel(DecodeArgs a)
+__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a)
 {
-    __shared__ float fac[kMaxMergeChunks];
-    __shared__ float s_m, s_l;
+    __shared__ float fac[kMaxMergeChunks], lsum[kMaxMergeChunks];
+    __shared__ float red[8];
     const int bh = blockIdx.x; // b * H + h
     const int b = bh / a.H, h = bh % a.H;
-    const int C = a.c, nc = a.n_chunks;
+    const int C = a.c, nc = a.n_chunks, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float *p0 = a.part + ((int64_t)b * nc * a.H + h) * (C + 2);
     const int64_t cstride = (int64_t)a.H * (C + 2);
-    if (threadIdx.x < 32) {
-        float mt = a.sink[h];
-        for (int j = threadIdx.x; j < nc; j += 32) mt = fmaxf(mt, p0[j * cstride]);
-        mt = warp_max(mt);
-        float lt = 0.f;
-        for (int j = threadIdx.x; j < nc; j += 32) {
-            const float mj = p0[j * cstride];
-            lt += (mj > -INFINITY) ? p0[j * cstride + 1] * __expf(mj - mt) : 0.f;
-        }
-        lt = warp_sum(lt);
-        if (mt > -INFINITY) lt += __expf(a.sink[h] - mt);
-        const float inv = (mt > -INFINITY && lt > 0.f) ? 1.f / lt : 0.f;
-        for (int j = threadIdx.x; j < nc; j += 32) {
-            const float mj = p0[j * cstride];
-            fac[j] = (mj > -INFINITY) ? __expf(mj - mt) * inv : 0.f;
-        }
-        if (threadIdx.x == 0) { s_m = mt; s_l = lt; }
+    // 1. every chunk's (max, sum) in one pass; block max
+    float mt = a.sink[h];
+    for (int j = tid; j < nc; j += 128) {
+        const float2 ml = *reinterpret_cast<const float2 *>(p0 + j * cstride);
+        fac[j] = ml.x;
+        lsum[j] = ml.y;
+        mt = fmaxf(mt, ml.x);
+    }
+    mt = warp_max(mt);
+    if (lane == 0) red[wid] = mt;
+    __syncthreads();
+    mt = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    // 2. the denominator: chunk sums rescaled to the common max, plus the sink
+    float lt = 0.f;
+    for (int j = tid; j < nc; j += 128) {
+        const float mj = fac[j];
+        lt += (mj > -INFINITY) ? lsum[j] * __expf(mj - mt) : 0.f;
+    }
+    lt = warp_sum(lt);
+    __syncthreads();
+    if (lane == 0) red[4 + wid] = lt;
+    __syncthreads();
+    lt = red[4] + red[5] + red[6] + red[7];
+    if (mt > -INFINITY) lt += __expf(a.sink[h] - mt);
+    const float inv = (mt > -INFINITY && lt > 0.f) ? 1.f / lt : 0.f;
+    for (int j = tid; j < nc; j += 128) {
+        const float mj = fac[j];
+        fac[j] = (mj > -INFINITY) ? __expf(mj - mt) * inv : 0.f;
     }
     __syncthreads();
-    for (int ch = threadIdx.x; ch < C; ch += blockDim.x) {
-        float acc = 0.f;
-        for (int j = 0; j < nc; ++j) // chunks without keys carry weight 0 and unwritten rows
-            if (fac[j] != 0.f) acc = fmaf(p0[j * cstride + 2 + ch], fac[j], acc);
-        a.o[(int64_t)bh * C + ch] = f32_to_bf16_bits(acc);
+    // 3. the weighted sum of the chunk outputs, two channels per thread and step
+    for (int ch = 2 * tid; ch < C; ch += 256) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int j = 0; j < nc; ++j) { // chunks without keys carry weight 0 and unwritten rows
+            const float f = fac[j];
+            if (f != 0.f) {
+                const float2 v = *reinterpret_cast<const float2 *>(p0 + j * cstride + 2 + ch);
+                acc.x = fmaf(v.x, f, acc.x);
+                acc.y = fmaf(v.y, f, acc.y);
+            }
+        }
+        *reinterpret_cast<uint32_t *>(a.o + (int64_t)bh * C + ch) =
+            uint32_t(f32_to_bf16_bits(acc.x)) | (uint32_t(f32_to_bf16_bits(acc.y)) << 16);
     }
-    if (a.lse && threadIdx.x == 0) a.lse[bh] = (s_m > -INFINITY) ? s_m + __logf(s_l) : -INFINITY;
+    if (a.lse && tid == 0) a.lse[bh] = (mt > -INFINITY) ? mt + __logf(lt) : -INFINITY;
 }
 
 template <int CPL>

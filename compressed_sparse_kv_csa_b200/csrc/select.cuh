@@ -2,9 +2,13 @@
 // order-preserving), shared by the top-k kernels.
 //
 // The keys of one selection usually share their leading bits (scores of one query lie within a few
-// binades), so the digits are taken from the bits that differ inside the block: keys are offset
-// by the block minimum and left-aligned on the highest bit of (max - min) before 8-bit digit
+// binades), so the digits are taken from the bits that differ inside the group: keys are offset
+// by the group minimum and left-aligned on the highest bit of (max - min) before 8-bit digit
 // passes.  The crossing bin of each pass is found by a warp suffix scan over the 256 bins.
+//
+// A selection runs on a group of NT threads (local ids 0..NT-1).  BAR = 0 synchronises the whole
+// block (__syncthreads, the group is the block); BAR > 0 uses named barrier BAR for a group that
+// is part of a block (e.g. the epilogue warps of a warp-specialised kernel).
 #pragma once
 
 #include <stdint.h>
@@ -38,25 +42,33 @@ template <typename K> __device__ __forceinline__ K warp_max_key(K v)
     return v;
 }
 
+template <int NT, int BAR> __device__ __forceinline__ void group_sync()
+{
+    if constexpr (BAR == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
 // Scratch in shared memory for block_kth.
 template <typename K> struct SelectSmem {
     int hist[256];
     K red[64];
     K kmin, kmax;
     int bin, rem;
+    int cnt[32];
+    uint32_t mn[32];
 };
 
 // Among the n keys get(i) (i < n), find thr = the k-th largest key (1 <= k <= n) and
-// n_gt = the number of keys strictly greater than thr.  All NT threads of the block call it and
-// all receive the result.
-template <int NT, typename K, typename Get>
-__device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int &n_gt)
+// n_gt = the number of keys strictly greater than thr.  All NT threads of the group call it (ltid =
+// the caller's id in the group) and all receive the result.
+template <int NT, typename K, int BAR = 0, typename Get>
+__device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int &n_gt, int ltid = threadIdx.x)
 {
     constexpr int KB = KeyBits<K>::bits;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int lane = ltid & 31, wid = ltid >> 5;
     // 1. range of the keys
     K lo = ~(K)0, hi = 0;
-    for (int i = tid; i < n; i += NT) {
+    for (int i = ltid; i < n; i += NT) {
         const K v = get(i);
         lo = v < lo ? v : lo;
         hi = v > hi ? v : hi;
@@ -64,8 +76,8 @@ __device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int 
     lo = warp_min_key(lo);
     hi = warp_max_key(hi);
     if (lane == 0) { sm->red[wid] = lo; sm->red[32 + wid] = hi; }
-    __syncthreads();
-    if (tid == 0) {
+    group_sync<NT, BAR>();
+    if (ltid == 0) {
         K a = sm->red[0], b = sm->red[32];
         for (int w = 1; w < NT / 32; ++w) {
             a = sm->red[w] < a ? sm->red[w] : a;
@@ -74,11 +86,12 @@ __device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int 
         sm->kmin = a;
         sm->kmax = b;
     }
-    __syncthreads();
+    group_sync<NT, BAR>();
     const K kmin = sm->kmin, range = sm->kmax - sm->kmin;
     if (range == 0) { // all keys equal
         thr = kmin;
         n_gt = 0;
+        group_sync<NT, BAR>(); // kmin / kmax are read before anyone reuses the scratch
         return;
     }
     const int lead = clz_key<K>(range);      // left-align the significant bits
@@ -88,13 +101,13 @@ __device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int 
     int rem = k;
     for (int p = 0; p < passes; ++p) {
         const int shift = KB - 8 * (p + 1);
-        for (int i = tid; i < 256; i += NT) sm->hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < n; i += NT) {
+        for (int i = ltid; i < 256; i += NT) sm->hist[i] = 0;
+        group_sync<NT, BAR>();
+        for (int i = ltid; i < n; i += NT) {
             const K r = (get(i) - kmin) << lead;
             if ((r & pmask) == prefix) atomicAdd(&sm->hist[(int)((r >> shift) & 255)], 1);
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         if (wid == 0) { // suffix scan from the top bin: lane l owns bins 255-8l .. 248-8l
             int c[8], s = 0;
 #pragma unroll
@@ -118,14 +131,61 @@ __device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int 
                 sm->rem = rem - cum;
             }
         }
-        __syncthreads();
+        group_sync<NT, BAR>();
         prefix |= (K)sm->bin << shift;
         pmask |= (K)255 << shift;
         rem = sm->rem;
-        __syncthreads();
+        group_sync<NT, BAR>();
     }
     thr = (prefix >> lead) + kmin;
     n_gt = k - rem;
+}
+
+// The k-th largest of n unique 64-bit keys (1 <= k <= n): a 32-bit radix selection on the high
+// words, then -- only when several keys share the threshold's high word and not all of them are
+// needed -- a second one on the low words of those ties.  Same calling rules as block_kth.
+template <int NT, int BAR = 0, typename Get>
+__device__ unsigned long long block_kth64(int n, int k, Get get, SelectSmem<uint32_t> *sm, int ltid = threadIdx.x)
+{
+    uint32_t thr_hi;
+    int n_gt;
+    block_kth<NT, uint32_t, BAR>(n, k, [&](int i) { return (uint32_t)(get(i) >> 32); }, sm, thr_hi, n_gt, ltid);
+    const int need = k - n_gt; // >= 1 keys with the threshold's high word
+    // count the ties and find their smallest low word
+    int cnt = 0;
+    uint32_t mn = 0xffffffffu;
+    for (int i = ltid; i < n; i += NT) {
+        const unsigned long long v = get(i);
+        if ((uint32_t)(v >> 32) == thr_hi) {
+            ++cnt;
+            mn = min(mn, (uint32_t)v);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    const int lane = ltid & 31, wid = ltid >> 5;
+    if (lane == 0) { sm->cnt[wid] = cnt; sm->mn[wid] = mn; }
+    group_sync<NT, BAR>();
+    int tot = 0;
+    uint32_t lo = 0xffffffffu;
+    for (int w = 0; w < NT / 32; ++w) {
+        tot += sm->cnt[w];
+        lo = min(lo, sm->mn[w]);
+    }
+    group_sync<NT, BAR>();
+    if (tot > need) { // select among the ties (non-ties map to 0, below every tie's low word)
+        uint32_t thr_lo;
+        int g;
+        block_kth<NT, uint32_t, BAR>(n, need, [&](int i) {
+            const unsigned long long v = get(i);
+            return (uint32_t)(v >> 32) == thr_hi ? (uint32_t)v : 0u;
+        }, sm, thr_lo, g, ltid);
+        lo = thr_lo;
+    }
+    return ((unsigned long long)thr_hi << 32) | lo;
 }
 
 } // namespace csa

@@ -175,6 +175,48 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     return d;
 }
 
+// 64-byte-swizzled K-major operand descriptor (rows of 64 bytes, 8-row atoms of 512 bytes):
+// SBO = byte stride between 8-row groups.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16; // LBO unused for swizzled K-major layouts
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61; // 64-byte swizzle
+    return d;
+}
+
+// Block-scaled MX FP4 (kind::mxf4, E2M1 A and B packed two per byte, E8M0 scales, one scale per
+// 32 elements of K, K = 64 per instruction): instruction descriptor.  Fields: B scale-factor id
+// [4,6), A format [7,10) and B format [10,13) (E2M1 = 1), A/B major [15]/[16] (K-major = 0),
+// N>>3 [17,23), scale format [23] (1 = E8M0), M>>4 [24,29), A scale-factor id [29,31), K size
+// [31] (0 = 64).  The scale-factor id selects the byte pair of the 32-bit TMEM scale word that
+// the instruction uses (0: bytes 0-1, 2: bytes 2-3).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sf_id_a, uint32_t sf_id_b)
+{
+    return (sf_id_b << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24) | (sf_id_a << 29);
+}
+
+// D[tmem] (+)= A * B with per-32-element E8M0 scales of A and B read from TMEM.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate));
+}
+
+// 32 lanes x 4 consecutive 32-bit columns: thread i of the warp writes lane (base + i).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+                 "r"(d));
+}
+
 // kind::f16 with f16 A and B (format code 0), f32 accumulate, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N)
 {

@@ -37,5 +37,22 @@ inline bool encode_bf16_rows(CUtensorMap *m, const void *base, uint64_t rows, ui
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rows of `row_bytes` bytes (row stride row_bytes) read as bytes in boxes of the whole row x
+// box_rows rows, with the 64-byte swizzle (row_bytes must be 64); rows outside read as zeros.
+// Used for packed FP4 operands (two E2M1 codes per byte, 64 bytes = 128 elements per row).
+inline bool encode_u8_rows_sw64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_bytes,
+                                uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+    if (!enc || rows == 0 || row_bytes != 64 || box_rows == 0 || box_rows > 256) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {row_bytes, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 } // namespace tma
 } // namespace csa

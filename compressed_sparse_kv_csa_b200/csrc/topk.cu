@@ -19,6 +19,7 @@ namespace {
 
 constexpr int TK_THREADS = 1024;
 constexpr int TK_MAX = 2048;
+constexpr int64_t TK_STAGE = 32768; // rows of at most this many scores are staged in shared memory
 
 __device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
 {
@@ -31,11 +32,15 @@ __device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
     return nv < 0 ? 0 : nv;
 }
 
+// STAGED: the row's scores (nv <= TK_STAGE) are first copied into shared memory as keys, so the
+// selection passes read shared memory instead of the score buffer.
+template <bool STAGED>
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
 {
     __shared__ unsigned long long sel[TK_MAX];
     __shared__ SelectSmem<uint32_t> ssel;
     __shared__ int s_cnt, s_warp[TK_THREADS / 32], s_eq_taken;
+    extern __shared__ uint32_t skeys[]; // STAGED only
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
@@ -43,20 +48,31 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     const int k = a.k;
     const int ke = (int)(nv < k ? nv : k);
     const float *S = a.scores + r * a.ld;
+    if (STAGED) { // rows are 16-byte aligned and padded to a multiple of 4 scores
+        for (int64_t i4 = tid; 4 * i4 < nv; i4 += TK_THREADS) {
+            const float4 v = *reinterpret_cast<const float4 *>(S + 4 * i4);
+            skeys[4 * i4 + 0] = float_key(v.x);
+            skeys[4 * i4 + 1] = float_key(v.y);
+            skeys[4 * i4 + 2] = float_key(v.z);
+            skeys[4 * i4 + 3] = float_key(v.w);
+        }
+        __syncthreads();
+    }
+    auto key = [&](int64_t i) { return STAGED ? skeys[i] : float_key(S[i]); };
 
     uint32_t thr = 0;   // k-th largest key (only meaningful when nv > k)
     int n_gt = 0;       // number of keys strictly above thr
     if (nv > k) {
-        block_kth<TK_THREADS, uint32_t>((int)nv, k, [&](int i) { return float_key(S[i]); }, &ssel, thr, n_gt);
+        block_kth<TK_THREADS, uint32_t>((int)nv, k, [&](int i) { return key(i); }, &ssel, thr, n_gt);
         const int rem = k - n_gt;
         if (tid == 0) { s_cnt = 0; s_eq_taken = 0; }
         __syncthreads();
         // strictly greater: unordered append
         for (int64_t s = tid; s < nv; s += TK_THREADS) {
-            const uint32_t key = float_key(S[s]);
-            if (key > thr) {
+            const uint32_t kv = key(s);
+            if (kv > thr) {
                 const int pos = atomicAdd(&s_cnt, 1);
-                if (pos < n_gt) sel[pos] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)s);
+                if (pos < n_gt) sel[pos] = ((unsigned long long)kv << 32) | (0xffffffffu - (uint32_t)s);
             }
         }
         __syncthreads();
@@ -65,7 +81,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
         for (int64_t base = 0; base < nv; base += TK_THREADS) {
             if (s_eq_taken >= need) break; // uniform: read after a barrier
             const int64_t s = base + tid;
-            const bool eq = (s < nv) && (float_key(S[s]) == thr);
+            const bool eq = (s < nv) && (key(s) == thr);
             const unsigned bal = __ballot_sync(0xffffffffu, eq);
             const int lane = tid & 31, wid = tid >> 5;
             if (lane == 0) s_warp[wid] = __popc(bal);
@@ -83,7 +99,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
         }
     } else {
         for (int64_t s = tid; s < nv; s += TK_THREADS)
-            sel[s] = ((unsigned long long)float_key(S[s]) << 32) | (0xffffffffu - (uint32_t)s);
+            sel[s] = ((unsigned long long)key(s) << 32) | (0xffffffffu - (uint32_t)s);
     }
     // bitonic sort (descending) of the ke winners, padded with zeros to a power of two
     int n2 = 1;
@@ -121,7 +137,14 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
 cudaError_t launch_topk(const IndexerArgs &a, cudaStream_t st)
 {
     if (a.Nq == 0) return cudaSuccess;
-    topk_kernel<<<(unsigned)a.Nq, TK_THREADS, 0, st>>>(a);
+    if (a.max_nvis <= TK_STAGE) {
+        const size_t smem = (size_t)((a.max_nvis + 3) / 4 * 4) * sizeof(uint32_t);
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        topk_kernel<true><<<(unsigned)a.Nq, TK_THREADS, smem, st>>>(a);
+    } else {
+        topk_kernel<false><<<(unsigned)a.Nq, TK_THREADS, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

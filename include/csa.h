@@ -49,8 +49,6 @@ extern "C" {
 /* device error word bits (csa_device_error) */
 #define CSA_DEVERR_TIMEOUT 1       /* a bounded wait ran out */
 #define CSA_DEVERR_INDEX 2         /* an out-of-range index was skipped */
-#define CSA_DEVERR_RANGE 4         /* FP4 decode indexer: a non-zero block scale outside 2^-23..2^13
-                                      met the exact-f16 tensor-core path; those scores are inexact */
 
 #define CSA_F32 0
 #define CSA_BF16 1
@@ -63,7 +61,8 @@ extern "C" {
  *   value[j] = e4m3(fp8[r, j]) * scale[r]        for j <  c - rope_dims
  *   value[j] = bf16(rope[r, j - (c-rope_dims)])  for j >= c - rope_dims
  * Planes: fp8 [n, c-rope_dims] bytes, rope [n, rope_dims] bf16 bits, scale [n] fp32.
- * Each plane base must be 16-byte aligned and (c - rope_dims) and rope_dims multiples of 16.
+ * The fp8 and rope plane bases must be 16-byte aligned, the scale plane 4-byte aligned, and
+ * (c - rope_dims) and rope_dims multiples of 16 (so any row range of a plane is a valid plane).
  */
 typedef struct csa_kv_rows {
     uint8_t *fp8;

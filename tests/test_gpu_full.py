@@ -6,6 +6,8 @@
   (block boundaries, random, last rows); attention on sampled rows with a seeded top-k list.
 * csa_decode_1m    (8 sequences at t = 1,048,576, 262,144 entries each): every sequence's FP4 key
   scan + top-k, and the attention of rows whose GPU and oracle top-k sets agree.
+* mixed_decode_64  (64 sequences, 4 stacked layers): three sampled sequences through every layer
+  and the glue, each GPU step checked on the oracle's inputs for that step.
 """
 import dataclasses
 
@@ -15,7 +17,7 @@ import torch
 
 import csa_workloads as WL
 import oracle as O
-from _util import check_topk, dev, host, row_rel_err
+from _util import check_fp4_near, check_topk, dev, host, row_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -218,64 +220,85 @@ def test_csa_decode_1m_full(C):
 
 
 def test_mixed_decode_64_stack_sampled(C):
-    """The stacked decode workload as the bench runs it (64 sequences, layers HCA, CSA, HCA, CSA,
-    glue between layers), checked on the shortest, a median and the longest sequence against the
-    oracle running the same stack from the same seeded inputs.  Layer outputs are stored in bf16
-    on both sides.  Each layer's output: 2e-2 max relative error per head row.  A CSA layer's
-    index query comes from the previous layer's output, so a few FP4 codes of it may sit on the
-    other side of a rounding boundary than the oracle's; its top-k set is therefore checked by
-    overlap (>= 95 %) and by every differing entry lying within 5 % of the oracle's k-th score."""
+    """The stacked decode workload as the bench builds it (64 sequences, layers HCA, CSA, HCA, CSA,
+    glue between layers), checked on the shortest, a median and the longest sequence.
+
+    The oracle runs the stack from the seeded inputs (layer outputs and next queries stored in
+    bf16, index queries in FP4, as on the GPU).  Each GPU layer is then checked on the oracle's
+    own inputs for that layer (oracle values fed to the GPU, never the reverse), so each check is
+    strict: top-k sets exact up to the 1e-4 tie band, attention outputs within 2e-2, glue as in
+    the glue parity test.  The bench's free-running GPU chain is checked for layer 0 (identical
+    inputs: strict) and, for the later layers, whose index queries are FP4 codes of slightly
+    different values, by top-k overlap >= 90 % and output error < 0.5 (an offset or wiring
+    mistake gives errors of order 1)."""
     import bench
     w = WL.WORKLOADS["mixed_decode_64"]
     job = bench.MixedDecode(w, 0, torch, C, torch.device("cuda", 0))
     job.step()
     torch.cuda.synchronize()
     assert C.csa_device_error() == 0
-    outs = [host(L.o) for L in job.layers]
-    idxs = [L.idx.cpu().numpy() if L.csa else None for L in job.layers]
+    chain_o = [host(L.o) for L in job.layers]
+    chain_idx = [L.idx.cpu().numpy() if L.csa else None for L in job.layers]
     H, c, Hi, di, W, k = w.H, w.c, w.H_I, w.d_I, w.W, w.k
     lens = job.lens
     order = np.argsort(lens)
     for b in (int(order[0]), int(order[len(order) // 2]), int(order[-1])):
         t = int(lens[b])
+        pos = torch.tensor([t], dtype=torch.int64, device="cuda")
+        wl1 = torch.tensor([W], dtype=torch.int32, device="cuda")
         q = WL.draw(w, "q", 0, 1, layer=0, seq=b).reshape(1, H, c).astype(np.float64)
         zi = None
         for l, L in enumerate(job.layers):
             m = L.m
             nv = (t + 1) // m
+            off = torch.tensor([int(L.off_np[b])], dtype=torch.int64, device="cuda")
+            win_b = C.KvRows(L.win.fp8[b * W:(b + 1) * W], L.win.rope[b * W:(b + 1) * W], L.win.scale[b * W:(b + 1) * W])
             f8, rb, sc = O.quant_kv(WL.draw(w, "WIN", 0, W, layer=l, seq=b))
             winrows = O.dequant_kv(f8, rb, sc)
             sink = WL.draw(w, "sink", 0, 1, layer=l)[0]
+            q_bf = dev(q.reshape(1, H, c).astype(np.float32), "bf16")
             if L.csa:
-                Qd = O.dequant_fp4(*O.quant_fp4(zi.astype(np.float32))).reshape(1, Hi, di)
+                qc, qs = O.quant_fp4(zi.astype(np.float32))
+                Qd = O.dequant_fp4(qc, qs).reshape(1, Hi, di)
                 wt = WL.draw(w, "w", 0, 1, layer=l, seq=b)
                 Kd = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "KI", 0, nv, layer=l, seq=b)))
                 idx_o, S = O.indexer_topk(Qd, wt, Kd, np.array([t]), m, k)
                 del Kd
-                g = idxs[l][b]
+                # GPU indexer on the oracle's index query (the same FP4 codes): strict
+                q4 = C.Fp4Rows(torch.from_numpy(qc).cuda(), torch.from_numpy(qs).cuda())
+                idx_g = C.indexer_topk(q4, dev(wt), L.keys, m, k, max_nvis=nv, q_pos=pos, key_off=off)
+                assert check_topk(idx_g.cpu().numpy(), idx_o, S, [nv], k) >= 0, (l, b)
+                # the free-running chain: overlap
                 ke = min(k, nv)
-                gs = g[:ke]
-                assert np.all(g[ke:] == -1) and np.all((gs >= 0) & (gs < nv)) and len(set(gs.tolist())) == ke
-                os_ = set(idx_o[0, :ke].tolist())
-                assert len(os_ & set(gs.tolist())) >= 0.95 * ke, (l, b, len(os_ & set(gs.tolist())))
-                kth = S[0, idx_o[0, ke - 1]]
-                for s in set(gs.tolist()) ^ os_:
-                    assert abs(S[0, s] - kth) <= 5e-2 * abs(kth), (l, b, s, S[0, s], kth)
+                g = chain_idx[l][b]
+                assert np.all(g[ke:] == -1) and len(set(g[:ke].tolist())) == ke
+                assert len(set(g[:ke].tolist()) & set(idx_o[0, :ke].tolist())) >= 0.9 * ke, (l, b)
                 sel = np.sort(idx_o[0, :ke])
                 f8, rb, sc = O.quant_kv(WL.draw(w, "KV", 0, nv, layer=l, seq=b)[sel])
                 comp = O.dequant_kv(f8, rb, sc)
-                remap = {int(s): j for j, s in enumerate(sel)}
-                loc = np.array([[remap[int(s)] for s in idx_o[0, :ke]] + [-1] * (k - ke)], np.int32)
+                remap = {int(s_): j for j, s_ in enumerate(sel)}
+                loc = np.array([[remap[int(s_)] for s_ in idx_o[0, :ke]] + [-1] * (k - ke)], np.int32)
                 o_ref, _ = O.hybrid_attn_decode(q, comp, [0], [t], winrows, [W], sink, 1.0, m, W, idx=loc)
+                o_g = C.hybrid_attn_decode(q_bf, L.comp, off, pos, win_b, wl1, dev(sink), 1.0, m, W, max_nvis=nv,
+                                           idx=torch.from_numpy(idx_o[:, :k].astype(np.int32)).cuda())
             else:
                 f8, rb, sc = O.quant_kv(WL.draw(w, "KV", 0, nv, layer=l, seq=b))
                 comp = O.dequant_kv(f8, rb, sc)
                 o_ref, _ = O.hybrid_attn_decode(q, comp, [0], [t], winrows, [W], sink, 1.0, m, W)
-            err = row_rel_err(outs[l][b:b + 1], o_ref)
+                o_g = C.hybrid_attn_decode(q_bf, L.comp, off, pos, win_b, wl1, dev(sink), 1.0, m, W, max_nvis=nv)
+            err = row_rel_err(host(o_g), o_ref)
             assert err.max() < 2e-2, (l, b, t, err.max())
+            chain_err = row_rel_err(chain_o[l][b:b + 1], o_ref).max()
+            assert chain_err < (2e-2 if l == 0 else 0.5), (l, b, t, chain_err)
             if l + 1 < len(job.layers):
                 o_b = O.bf16_value(O.bf16_bits(o_ref.reshape(H, c)))        # layer output stored in bf16
                 P = WL.draw(w, "P", 0, c, layer=l)
                 Rm = WL.draw(w, "Rm", 0, di, layer=l)
                 qn, zi = O.decode_glue(o_b, P, Rm)
+                # GPU glue on the oracle's layer output: strict
+                qn_g, qI_g = C.csa_decode_glue(dev(o_b.astype(np.float32), "bf16"), L.P, L.Rm)
+                assert row_rel_err(host(qn_g), qn).max() <= 5e-3
+                if qI_g is not None:
+                    check_fp4_near(qI_g.codes.cpu().numpy(), qI_g.scales.cpu().numpy(), zi)
                 q = O.bf16_value(O.bf16_bits(qn)).reshape(1, H, c).astype(np.float64)
+    assert C.csa_device_error() == 0

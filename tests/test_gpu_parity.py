@@ -192,12 +192,44 @@ def test_indexer_topk_fp4_decode_batches(C):
     assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
 
 
-def test_fp4_decode_topk_ties_across_chunks(C):
+@pytest.mark.parametrize("Bn,k", [(16, 1024), (12, 2048)])
+def test_fp4_decode_streaming_filter(C, Bn, k):
+    """Chunks longer than the scan's candidate buffer (16 or 12 sequences of 40-60k entries), so
+    the streaming filter cuts its buffer back to the k best and raises its bar mid-chunk."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    H, d, m = 64, 128, 4
+    g = np.random.default_rng(Bn)
+    nv = g.integers(40000, 60000, size=Bn).astype(np.int64)
+    pos = nv * m + g.integers(0, m, size=Bn)
+    off = np.concatenate([[3], 3 + np.cumsum(nv)[:-1]]).astype(np.int64)
+    keys = np.concatenate([np.zeros((3, d), np.float32)] +
+                          [WL.draw(w, "KI", 0, int(n), seq=100 + b) for b, n in enumerate(nv)])
+    qx = np.stack([WL.draw(w, "qI", 0, 1, seq=100 + b).reshape(H, d) for b in range(Bn)])
+    wt = np.concatenate([WL.draw(w, "w", 0, 1, seq=100 + b) for b in range(Bn)])
+    kc, ks = O.quant_fp4(keys)
+    qc, qs = O.quant_fp4(qx.reshape(Bn * H, d))
+    Kd = O.dequant_fp4(kc, ks)
+    Qd = O.dequant_fp4(qc, qs).reshape(Bn, H, d)
+    idx_o, S = O.indexer_topk(Qd, wt, Kd, pos, m, k, kbase=off)
+    k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
+    q4 = C.Fp4Rows.empty(Bn * H, d, "cuda")
+    C.csa_quantize_fp4(dev(keys), k4)
+    C.csa_quantize_fp4(dev(qx.reshape(Bn * H, d)), q4)
+    idx = C.indexer_topk(q4, dev(wt), k4, m, k, max_nvis=int(nv.max()),
+                         q_pos=torch.from_numpy(pos).cuda(), key_off=torch.from_numpy(off).cuda())
+    torch.cuda.synchronize()
+    assert C.csa_device_error() == 0
+    assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
+
+
+@pytest.mark.parametrize("Bn,n0", [(2, 40000), (16, 45000)])
+def test_fp4_decode_topk_ties_across_chunks(C, Bn, n0):
     """All scores equal (q = 0): every query keeps the lowest k entries, which requires the
-    per-chunk selections and their merge to break ties by entry index."""
-    Bn, H, d, k = 2, 64, 128, 1024
-    nv = np.array([40000, 700], np.int64)
-    off = np.array([5, 40005], np.int64)
+    per-chunk selections (and, with 16 sequences, the scan's mid-chunk buffer cuts) and their
+    merge to break ties by entry index."""
+    H, d, k = 64, 128, 1024
+    nv = np.array([n0] * (Bn - 1) + [700], np.int64)
+    off = 5 + np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
     g = np.random.default_rng(9)
     keys = g.standard_normal((int(off[-1] + nv[-1]), d)).astype(np.float32)
     k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
@@ -208,8 +240,9 @@ def test_fp4_decode_topk_ties_across_chunks(C):
     idx = C.indexer_topk(q4, torch.ones((Bn, H), device="cuda"), k4, 4, k, max_nvis=int(nv.max()),
                          q_pos=torch.from_numpy(nv * 4 - 1).cuda(), key_off=torch.from_numpy(off).cuda(), score_out=sc)
     ig = idx.cpu().numpy()
-    assert list(ig[0]) == list(range(k))
-    assert list(ig[1]) == list(range(700)) + [-1] * (k - 700)
+    for b in range(Bn - 1):
+        assert list(ig[b]) == list(range(k))
+    assert list(ig[Bn - 1]) == list(range(700)) + [-1] * (k - 700)
     assert np.all(sc.cpu().numpy()[idx.cpu().numpy() >= 0] == 0.0)
 
 

@@ -1,0 +1,62 @@
+"""Host logic of the multi-GPU bench, run as two CPU processes over the gloo backend.
+
+The workloads shard by whole problems (layers, sequences): each rank draws its own sequences and
+the ranks exchange nothing but the timing reduction.  These tests check that reduction (the
+job's time is the slowest rank's, identical on every rank) and that the ranks' seeded inputs are
+disjoint and of equal size.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        import csa_workloads as WL
+        out = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.25 * rank], world, dist, torch.device("cpu"))
+        w = WL.WORKLOADS["csa_decode_1m"]
+        seqs = bench.rank_sequences(w.B, rank)
+        first_rows = np.stack([WL.draw(w, "KI", 0, 2, seq=s)[0] for s in seqs])
+        dist.barrier()
+        q.put((rank, out, seqs, first_rows))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_timing_reduction_and_disjoint_shards():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=120) for _ in range(2)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, out0, s0, rows0), (r1, out1, s1, rows1) = res
+    assert out0 == out1 == [2.0, 10.0, 0.25]        # element-wise max, the same on every rank
+    assert len(s0) == len(s1) and not set(s0) & set(s1)  # equal shares, no shared sequence
+    assert not np.array_equal(rows0, rows1)
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.max_over_ranks([3.0, 4.0], 1, None, None) == [3.0, 4.0]
+    assert bench.rank_sequences(4, 0) == [0, 1, 2, 3]
+    assert bench.rank_sequences(4, 2) == [8, 9, 10, 11]
