@@ -7,7 +7,9 @@
 // concatenated); KV cache with BF16 RoPE dims and FP8 for the rest ("Mind Observatory: Uncovering
 // the technical ledger of DeepSeek-V4"); the per-head sink is folded in by the merge kernel.
 //
-// Grid = (chunks of 128 keys, sequences).  Each CTA:
+// Work items = (sequence, chunk of 128 keys of its key list); persistent CTAs (one per SM) walk
+// the items, so the many empty chunks of short sequences in a mixed batch cost no launch.  For each
+// non-empty item a CTA:
 //   1. stages q [64 x 512] (bf16) and gathers its 128 key rows -- window rows first, then the
 //      top-k (CSA) or visible (HCA) compressed rows -- dequantising the FP8 part (code x row scale)
 //      to bf16 next to the BF16 RoPE part, all in 128-byte-swizzled shared memory;
@@ -33,7 +35,9 @@ constexpr uint32_t OFF_K = 65536;    // 8 sub-tiles [128 x 128 B]  128 KB
 constexpr uint32_t OFF_P = 196608;   // 2 sub-tiles [64 x 128 B]   16 KB
 constexpr uint32_t OFF_VALID = 212992; // 128 flags
 constexpr uint32_t OFF_ROWS = OFF_VALID + 512; // 128 resolved key rows (int64)
-constexpr uint32_t OFF_BAR = OFF_ROWS + 1024;
+constexpr int kSeqCache = 1024;                  // per-sequence key counts kept in shared memory
+constexpr uint32_t OFF_SEQ = OFF_ROWS + 1024;    // n_win [kSeqCache], n_keys [kSeqCache] (int32)
+constexpr uint32_t OFF_BAR = OFF_SEQ + 8 * kSeqCache;
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = OFF_TMEM + 64 + 1024;
 constexpr uint32_t TMEM_O = 16u << 16;
@@ -88,25 +92,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
     const uint32_t bar_s = base + OFF_BAR, bar_o = base + OFF_BAR + 8, bar_f = base + OFF_BAR + 16;
     int *valid = reinterpret_cast<int *>(sp + OFF_VALID);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.y, chunk = blockIdx.x;
-    const int n_win = a.win_len[b] < 0 ? 0 : (a.win_len[b] > a.W ? a.W : a.win_len[b]);
-    int64_t n_cmp;
-    if (a.idx) n_cmp = a.k;
-    else {
-        n_cmp = (a.pos[b] + 1) / a.m;
-        if (n_cmp > a.max_nvis) n_cmp = a.max_nvis;
-        if (n_cmp < 0) n_cmp = 0;
-    }
-    const int64_t n_keys = n_win + n_cmp;
-    const int64_t j0 = (int64_t)chunk * kKT;
-    float *part = a.part + ((int64_t)b * a.n_chunks + chunk) * kH * (kC + 2);
-    if (j0 >= n_keys) { // empty chunk: a neutral partial (CTA-uniform exit)
-        for (int h = tid; h < kH; h += kThreads) {
-            part[(int64_t)h * (kC + 2)] = -INFINITY;
-            part[(int64_t)h * (kC + 2) + 1] = 0.f;
-        }
-        return;
-    }
     if (tid == 0) {
         mbar_init(bar_s, 1);
         mbar_init(bar_o, 1);
@@ -114,188 +99,239 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
         mbar_init_fence();
     }
     if (warp == kMmaWarp) tmem_alloc(base + OFF_TMEM, 512);
-
-    // ---- resolve the chunk's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
-    int64_t *rows = reinterpret_cast<int64_t *>(sp + OFF_ROWS);
-    if (tid < kKT) {
-        const int64_t j = j0 + tid;
-        int64_t code = -1;
-        if (j < n_keys && j < n_win) {
-            code = (int64_t)b * a.W + j;
-        } else if (j < n_keys) {
-            const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
-            if (s >= 0) {
-                const int64_t r = a.comp_off[b] + s;
-                if (r >= 0 && r < a.comp.n) code = r | (1ll << 62);
-                else flag_error(a.err, CSA_DEVERR_INDEX);
-            }
-        }
-        rows[tid] = code;
-        valid[tid] = code >= 0 ? 1 : 0;
-    }
-    // ---- stage q (all threads): 16 independent 16-byte loads per thread in flight
-    for (int e0 = tid; e0 < kH * (kC / 8); e0 += 16 * kThreads) {
-        uint4 v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int e = e0 + u * kThreads;
-            if (e < kH * (kC / 8))
-                v[u] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + (e >> 6)) * kC + 8 * (e & 63)));
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int e = e0 + u * kThreads;
-            if (e < kH * (kC / 8)) {
-                const int h = e >> 6, cc = e & 63;
-                sts4(sQ + (uint32_t)(cc >> 3) * 8192u + sw128_off(h, (cc & 7) * 8), v[u]);
-            }
-        }
-    }
-    __syncthreads();
-    // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as is;
-    // 12 independent loads per thread in flight
-    const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
-    constexpr int kU = 12;
-    for (int e0 = tid; e0 < kKT * (kC / 8); e0 += kU * kThreads) {
-        uint4 raw[kU];
-        float sc[kU];
-        int kind[kU]; // 0 empty, 1 FP8, 2 RoPE
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int e = e0 + u * kThreads;
-            kind[u] = 0;
-            raw[u] = make_uint4(0, 0, 0, 0);
-            sc[u] = 0.f;
-            if (e < kKT * (kC / 8)) {
-                const int64_t code = rows[e >> 6];
-                if (code >= 0) {
-                    const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
-                    const int64_t row = code & ((1ll << 62) - 1);
-                    const int ch = 8 * (e & 63);
-                    if (ch < cn) {
-                        const uint2 c = __ldg(reinterpret_cast<const uint2 *>(kv.fp8 + row * cn + ch));
-                        raw[u].x = c.x;
-                        raw[u].y = c.y;
-                        sc[u] = __ldg(kv.scale + row);
-                        kind[u] = 1;
-                    } else {
-                        raw[u] = __ldg(reinterpret_cast<const uint4 *>(kv.rope + row * kv.rope_dims + (ch - cn)));
-                        kind[u] = 2;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int e = e0 + u * kThreads;
-            if (e < kKT * (kC / 8)) {
-                const int jj = e >> 6, cc = e & 63;
-                const uint4 v = kind[u] == 1 ? fp8x8_to_bf16(make_uint2(raw[u].x, raw[u].y), sc[u]) : raw[u];
-                sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
-            }
-        }
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + OFF_TMEM);
-    bool ok = true;
-
-    if (warp == kMmaWarp && lane == 0) { // S = Q K^T
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + kColS, sdesc_sw128(sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024),
-                         sdesc_sw128(sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024), IDESC_S, (s | kk) != 0);
-        mma_commit(bar_s);
+    // window length and key count of every sequence, read once (the items loop checks them often)
+    int *s_nwin = reinterpret_cast<int *>(sp + OFF_SEQ), *s_nkeys = s_nwin + kSeqCache;
+    auto seq_counts = [&](int b, int &nw, int64_t &nk) {
+        nw = a.win_len[b] < 0 ? 0 : (a.win_len[b] > a.W ? a.W : a.win_len[b]);
+        int64_t nc;
+        if (a.idx) nc = a.k;
+        else {
+            nc = (a.pos[b] + 1) / a.m;
+            if (nc > a.max_nvis) nc = a.max_nvis;
+            if (nc < 0) nc = 0;
+        }
+        nk = nw + nc;
+    };
+    for (int b = tid; b < a.B && b < kSeqCache; b += kThreads) {
+        int nw;
+        int64_t nk;
+        seq_counts(b, nw, nk);
+        s_nwin[b] = nw;
+        s_nkeys[b] = (int)nk;
     }
-    const bool upper = lane < 16;
-    const int row = 16 * (warp & 3) + (lane & 15);
-    if (warp < 4) { // softmax of the chunk: lane l keys 0-63, lane l+16 keys 64-127 of head `row`
-        const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_s, 0));
-        if (ok) {
-            tc_fence_after();
-            uint32_t r0[32], r1[32], r2[32], r3[32];
-            tmem_ld32(tw + kColS, r0);
-            tmem_ld32(tw + kColS + 32, r1);
-            tmem_ld32(tw + kColS + 64, r2);
-            tmem_ld32(tw + kColS + 96, r3);
-            tmem_ld_wait();
-            float sv[64];
-            const int kb = upper ? 0 : 64;
-            const float sl2 = a.scale * kLog2e;
-            float mt = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
-                const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
-                float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
-                s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
-                s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
-                sv[e] = s0;
-                sv[32 + e] = s1;
-                mt = fmaxf(mt, fmaxf(s0, s1));
+    __syncthreads();
+    const int64_t n_items = (int64_t)a.B * a.n_chunks;
+    uint32_t ph = 0; // parity of bar_s / bar_o for the next non-empty item
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int b = (int)(item / a.n_chunks), chunk = (int)(item % a.n_chunks);
+        int n_win;
+        int64_t n_keys;
+        if (b < kSeqCache) {
+            n_win = s_nwin[b];
+            n_keys = s_nkeys[b];
+        } else {
+            seq_counts(b, n_win, n_keys);
+        }
+        const int64_t j0 = (int64_t)chunk * kKT;
+        float *part = a.part + ((int64_t)b * a.n_chunks + chunk) * kH * (kC + 2);
+        if (j0 >= n_keys) { // empty chunk: a neutral partial (CTA-uniform)
+            for (int h = tid; h < kH; h += kThreads) {
+                part[(int64_t)h * (kC + 2)] = -INFINITY;
+                part[(int64_t)h * (kC + 2) + 1] = 0.f;
             }
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-            float ls = 0.f;
-#pragma unroll
-            for (int e = 0; e < 64; ++e) {
-                const float p = (mt == -INFINITY) ? 0.f : ex2(sv[e] - mt);
-                sv[e] = p;
-                ls += p;
+            continue;
+        }
+
+        // ---- resolve the chunk's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
+        int64_t *rows = reinterpret_cast<int64_t *>(sp + OFF_ROWS);
+        if (tid < kKT) {
+            const int64_t j = j0 + tid;
+            int64_t code = -1;
+            if (j < n_keys && j < n_win) {
+                code = (int64_t)b * a.W + j;
+            } else if (j < n_keys) {
+                const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
+                if (s >= 0) {
+                    const int64_t r = a.comp_off[b] + s;
+                    if (r >= 0 && r < a.comp.n) code = r | (1ll << 62);
+                    else flag_error(a.err, CSA_DEVERR_INDEX);
+                }
             }
-            ls += __shfl_xor_sync(0xffffffffu, ls, 16);
-            const uint32_t psub = sP + (uint32_t)(kb >> 6) * 8192u;
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-                sts4(psub + sw128_off(row, 8 * g),
-                     make_uint4(pk_bf16(sv[8 * g], sv[8 * g + 1]), pk_bf16(sv[8 * g + 2], sv[8 * g + 3]),
-                                pk_bf16(sv[8 * g + 4], sv[8 * g + 5]), pk_bf16(sv[8 * g + 6], sv[8 * g + 7])));
-            if (upper) {
-                part[(int64_t)row * (kC + 2)] = (mt == -INFINITY) ? -INFINITY : mt * kLn2; // natural-log max
-                part[(int64_t)row * (kC + 2) + 1] = ls;
+            rows[tid] = code;
+            valid[tid] = code >= 0 ? 1 : 0;
+        }
+        // ---- stage q (all threads): 16 independent 16-byte loads per thread in flight
+        for (int e0 = tid; e0 < kH * (kC / 8); e0 += 16 * kThreads) {
+            uint4 v[16];
+    #pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < kH * (kC / 8))
+                    v[u] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + (e >> 6)) * kC + 8 * (e & 63)));
+            }
+    #pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < kH * (kC / 8)) {
+                    const int h = e >> 6, cc = e & 63;
+                    sts4(sQ + (uint32_t)(cc >> 3) * 8192u + sw128_off(h, (cc & 7) * 8), v[u]);
+                }
+            }
+        }
+        __syncthreads();
+        // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as is;
+        // 12 independent loads per thread in flight
+        const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
+        constexpr int kU = 12;
+        for (int e0 = tid; e0 < kKT * (kC / 8); e0 += kU * kThreads) {
+            uint4 raw[kU];
+            float sc[kU];
+            int kind[kU]; // 0 empty, 1 FP8, 2 RoPE
+    #pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int e = e0 + u * kThreads;
+                kind[u] = 0;
+                raw[u] = make_uint4(0, 0, 0, 0);
+                sc[u] = 0.f;
+                if (e < kKT * (kC / 8)) {
+                    const int64_t code = rows[e >> 6];
+                    if (code >= 0) {
+                        const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
+                        const int64_t row = code & ((1ll << 62) - 1);
+                        const int ch = 8 * (e & 63);
+                        if (ch < cn) {
+                            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(kv.fp8 + row * cn + ch));
+                            raw[u].x = c.x;
+                            raw[u].y = c.y;
+                            sc[u] = __ldg(kv.scale + row);
+                            kind[u] = 1;
+                        } else {
+                            raw[u] = __ldg(reinterpret_cast<const uint4 *>(kv.rope + row * kv.rope_dims + (ch - cn)));
+                            kind[u] = 2;
+                        }
+                    }
+                }
+            }
+    #pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int e = e0 + u * kThreads;
+                if (e < kKT * (kC / 8)) {
+                    const int jj = e >> 6, cc = e & 63;
+                    const uint4 v = kind[u] == 1 ? fp8x8_to_bf16(make_uint2(raw[u].x, raw[u].y), sc[u]) : raw[u];
+                    sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
+                }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-    }
-    __syncthreads();
-    ok = __syncthreads_and(ok);
-    if (warp == kMmaWarp && lane == 0 && ok) { // O = P V
+        __syncthreads();
         tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16(h ? tmem : tmem + TMEM_O,
-                         sdesc_sw128(sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024),
-                         sdesc_sw128(sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024), IDESC_PV, kk > 0);
-        mma_commit(bar_o);
-    }
-    if (warp < 4 && ok) { // unnormalised O rows -> workspace (lane l: channels 256-511, l+16: 0-255)
-        const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-        if (__all_sync(0xffffffffu, mbar_wait(bar_o, 0))) {
-            tc_fence_after();
-            float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
-            for (int c = 0; c < 8; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tw + 32u * c, r);
-                tmem_ld_wait();
-                // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
-                // 8-byte stores are the widest that are aligned for every row
-#pragma unroll
-                for (int g = 0; g < 16; ++g)
-                    *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
-                        make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
-            }
-        } else {
-            ok = false;
+
+        if (warp == kMmaWarp && lane == 0) { // S = Q K^T
+    #pragma unroll
+            for (int s = 0; s < 8; ++s)
+    #pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + kColS, sdesc_sw128(sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024),
+                             sdesc_sw128(sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024), IDESC_S, (s | kk) != 0);
+            mma_commit(bar_s);
         }
+        const bool upper = lane < 16;
+        const int row = 16 * (warp & 3) + (lane & 15);
+        if (warp < 4) { // softmax of the chunk: lane l keys 0-63, lane l+16 keys 64-127 of head `row`
+            const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_s, ph));
+            if (ok) {
+                tc_fence_after();
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tw + kColS, r0);
+                tmem_ld32(tw + kColS + 32, r1);
+                tmem_ld32(tw + kColS + 64, r2);
+                tmem_ld32(tw + kColS + 96, r3);
+                tmem_ld_wait();
+                float sv[64];
+                const int kb = upper ? 0 : 64;
+                const float sl2 = a.scale * kLog2e;
+                float mt = -INFINITY;
+    #pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
+                    const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
+                    float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
+                    s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
+                    s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
+                    sv[e] = s0;
+                    sv[32 + e] = s1;
+                    mt = fmaxf(mt, fmaxf(s0, s1));
+                }
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                float ls = 0.f;
+    #pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const float p = (mt == -INFINITY) ? 0.f : ex2(sv[e] - mt);
+                    sv[e] = p;
+                    ls += p;
+                }
+                ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+                const uint32_t psub = sP + (uint32_t)(kb >> 6) * 8192u;
+    #pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    sts4(psub + sw128_off(row, 8 * g),
+                         make_uint4(pk_bf16(sv[8 * g], sv[8 * g + 1]), pk_bf16(sv[8 * g + 2], sv[8 * g + 3]),
+                                    pk_bf16(sv[8 * g + 4], sv[8 * g + 5]), pk_bf16(sv[8 * g + 6], sv[8 * g + 7])));
+                if (upper) {
+                    part[(int64_t)row * (kC + 2)] = (mt == -INFINITY) ? -INFINITY : mt * kLn2; // natural-log max
+                    part[(int64_t)row * (kC + 2) + 1] = ls;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+        }
+        __syncthreads();
+        ok = __syncthreads_and(ok);
+        if (warp == kMmaWarp && lane == 0 && ok) { // O = P V
+            tc_fence_after();
+    #pragma unroll
+            for (int h = 0; h < 2; ++h)
+    #pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(h ? tmem : tmem + TMEM_O,
+                             sdesc_sw128(sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024),
+                             sdesc_sw128(sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024), IDESC_PV, kk > 0);
+            mma_commit(bar_o);
+        }
+        if (warp < 4 && ok) { // unnormalised O rows -> workspace (lane l: channels 256-511, l+16: 0-255)
+            const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+            if (__all_sync(0xffffffffu, mbar_wait(bar_o, ph))) {
+                tc_fence_after();
+                float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tw + 32u * c, r);
+                    tmem_ld_wait();
+                    // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
+                    // 8-byte stores are the widest that are aligned for every row
+    #pragma unroll
+                    for (int g = 0; g < 16; ++g)
+                        *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
+                            make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
+                }
+            } else {
+                ok = false;
+            }
+            tc_fence_before();
+        }
+        // the item's TMEM and shared memory are free once every warp is past this point
         tc_fence_before();
-    }
+        ok = __syncthreads_and(ok);
+        tc_fence_after();
+        ph ^= 1;
+    } // items
     if (!ok && tid == 0) flag_error(a.err, CSA_DEVERR_TIMEOUT);
     if (warp == kMmaWarp && lane == 0) {
         mma_commit(bar_f);
@@ -322,7 +358,14 @@ cudaError_t launch_attn_decode_tc(const DecodeArgs &a, cudaStream_t st)
     cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    decode_attn_tc_kernel<<<dim3((unsigned)a.n_chunks, (unsigned)a.B), kThreads, SMEM_ALLOC, st>>>(a);
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t items = (int64_t)a.B * a.n_chunks;
+    const int64_t grid = items < sms ? items : sms;
+    decode_attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(a);
     return cudaGetLastError();
 }
 

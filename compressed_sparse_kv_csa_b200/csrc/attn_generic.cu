@@ -276,8 +276,23 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a)
     __shared__ float red[8];
     const int bh = blockIdx.x; // b * H + h
     const int b = bh / a.H, h = bh % a.H;
-    const int C = a.c, nc = a.n_chunks, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const float *p0 = a.part + ((int64_t)b * nc * a.H + h) * (C + 2);
+    const int C = a.c, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // only the chunks that hold keys of this sequence (the rest carry weight 0)
+    int64_t n_keys;
+    {
+        const int nw = a.win_len[b] < 0 ? 0 : (a.win_len[b] > a.W ? a.W : a.win_len[b]);
+        int64_t ncmp;
+        if (a.idx) ncmp = a.k;
+        else {
+            ncmp = (a.pos[b] + 1) / a.m;
+            if (ncmp > a.max_nvis) ncmp = a.max_nvis;
+            if (ncmp < 0) ncmp = 0;
+        }
+        n_keys = nw + ncmp;
+    }
+    const int nc_all = a.n_chunks;
+    const int nc = (int)min((int64_t)nc_all, (n_keys + a.chunk - 1) / a.chunk);
+    const float *p0 = a.part + ((int64_t)b * nc_all * a.H + h) * (C + 2);
     const int64_t cstride = (int64_t)a.H * (C + 2);
     // 1. every chunk's (max, sum) in one pass; block max
     float mt = a.sink[h];

@@ -21,8 +21,10 @@
 //     is rescaled in TMEM) only when a tile raises it by more than 8.
 //   * Keys per token: tile 0 = window rows t-127..t of x_win; then tiles of 128 compressed rows
 //     (every visible entry for HCA, the top-k list for CSA).  Invalid slots are zero-filled and
-//     masked.  Keys are gathered by four producer warps into 128-byte-swizzled shared memory
-//     (two halves of 256 channels, each released as soon as its half of P V has consumed it).
+//     masked.  Window and HCA tiles are contiguous rows (2-D TMA boxes); CSA tiles are gathered
+//     through the top-k list with TMA gather4 (4 rows x 64 channels per instruction, one per
+//     producer thread and half tile).  Both land 128-byte-swizzled in two halves of 256 channels,
+//     each released as soon as its half of P V has consumed it.
 //   * Roles: warps 0-3 softmax / rescale / epilogue, warps 4-7 producers, warp 8 TMEM allocation
 //     and (one lane) MMA issue.  Every wait is an mbarrier wait bounded by %globaltimer; a wait
 //     that runs out records CSA_DEVERR_TIMEOUT and the CTA winds down without trapping.
@@ -89,11 +91,6 @@ __device__ __forceinline__ const uint16_t *key_row(const PrefillArgs &a, int64_t
     return (const uint16_t *)a.kv_comp + s * kC;
 }
 
-__device__ __forceinline__ uint4 ldg16(const uint16_t *p)
-{
-    return __ldg(reinterpret_cast<const uint4 *>(p));
-}
-
 __device__ __forceinline__ void sts16(uint32_t addr, uint4 v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -122,10 +119,25 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity)
 }
 
 // Tensor maps of q viewed as [T*64, 512], of x_win [T, 512] and of kv_comp [n_comp, 512], all
-// bf16 with 64-channel boxes and 128-byte swizzle (rows: 64 for q, 128 for keys).
+// bf16 with 64-channel boxes and 128-byte swizzle (rows: 64 for q, 128 for keys, 1 for the
+// gather map of kv_comp).
 struct TmaMaps {
-    CUtensorMap q, x, kv;
+    CUtensorMap q, x, kv, kvg;
 };
+
+// Compressed row of slot j of CSA tile i for token t, or -1 when the slot is empty or invalid.
+__device__ __forceinline__ int32_t gather_row(const PrefillArgs &a, int64_t t, int i, int j, int64_t n_cmp,
+                                              bool report)
+{
+    const int64_t slot = (int64_t)(i - 1) * kKT + j;
+    if (slot >= n_cmp) return -1;
+    const int32_t s = a.idx[t * a.k + slot];
+    if (s >= a.n_comp) {
+        if (report) flag_error(a.err, CSA_DEVERR_INDEX);
+        return -1;
+    }
+    return s;
+}
 
 struct Smem {
     uint32_t sQ, sK, sP, bars;
@@ -315,21 +327,18 @@ __device__ __forceinline__ bool producer_role(const PrefillArgs &a, const TmaMap
                     }
                     continue;
                 }
-                // gathered half h: 128 keys x 256 channels; thread owns chunk cc of keys j0 + 4*it
-                const int cc = ptid & 31, j0 = ptid >> 5;
-                const uint32_t dsub = dst + (uint32_t)(cc >> 3) * 16384u;
-                for (int it0 = 0; it0 < 32; it0 += 16) {
-                    uint4 v[16];
+                // gathered half h: 128 keys x 256 channels; thread = (4-key group g, 64-channel box q)
+                // issues one gather4 of 512 bytes; empty slots read row 0 and are masked
+                const int g = ptid >> 2, q = ptid & 3;
+                int32_t rr[4];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const uint16_t *rp = key_row(a, t, i, j0 + 4 * (it0 + u), n_cmp, h == 0 && cc == 0);
-                        v[u] = rp ? ldg16(rp + 256 * h + 8 * cc) : make_uint4(0, 0, 0, 0);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) sts16(dsub + sw128_off(j0 + 4 * (it0 + u), (cc & 7) * 8), v[u]);
+                for (int u = 0; u < 4; ++u) {
+                    const int32_t s = gather_row(a, t, i, 4 * g + u, n_cmp, h == 0 && q == 0);
+                    rr[u] = s < 0 ? 0 : s;
                 }
-                fence_proxy_async_smem();
-                mbar_arrive(S.bar(B_KVFULL0 + h));
+                mbar_arrive_expect_tx(S.bar(B_KVFULL0 + h), 512u);
+                tma_gather4(dst + (uint32_t)q * 16384u + (uint32_t)(4 * g) * 128u, &M.kvg, 256 * h + 64 * q, rr[0],
+                            rr[1], rr[2], rr[3], S.bar(B_KVFULL0 + h));
             }
         }
     }
@@ -437,7 +446,8 @@ cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *
     if (!encode_rows512(&maps.q, a.q, (uint64_t)a.T * kH, 64) || !encode_rows512(&maps.x, a.x_win, (uint64_t)a.T, kKT))
         return cudaSuccess; // no tensor-map encoder: the generic path serves the call
     const bool have_kv = a.kv_comp != nullptr && a.n_comp > 0;
-    if (!encode_rows512(&maps.kv, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, kKT))
+    if (!encode_rows512(&maps.kv, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, kKT) ||
+        !encode_rows512(&maps.kvg, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, 1))
         return cudaSuccess;
     *handled = true;
     int dev = 0, sms = 0;

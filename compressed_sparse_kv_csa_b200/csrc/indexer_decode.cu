@@ -14,15 +14,14 @@
 // up to 16,384 keys in 128-key tiles through an 8-stage ring:
 //   * producer warp: one lane issues the TMA load of the tile's codes (128 rows x 64 bytes,
 //     64-byte swizzle, the MMA's K-major layout); the 32 lanes copy the tile's scale words
-//     (4 bytes per key) with cp.async;
-//   * 4 scale warps (one per TMEM lane quadrant): write the tile's scale words into the TMEM
-//     scale-factor columns of its stage (query scales once at the start);
-//   * MMA lane: two M=128 (keys) x N=64 (heads) x K=64 block-scaled MMAs per tile into one of
-//     four TMEM accumulators;
+//     (4 bytes per key) with cp.async into the 32-row x 16-byte block the scale-factor copy
+//     reads (row l holds the words of keys l, l+32, l+64, l+96);
+//   * MMA lane: copies the tile's scale words into TMEM (tcgen05.cp 32x128b.warpx4), then two
+//     M=128 (keys) x N=64 (heads) x K=64 block-scaled MMAs into one of four TMEM accumulators;
 //   * 4 epilogue warps (one key per lane): score = w . ReLU(row of 64 head dot products), then a
 //     streaming filter: a key enters the chunk's candidate buffer only if it beats the current
-//     k-th best; when the buffer fills, an exact radix selection cuts it back to k and raises
-//     the bar.  At the end the chunk's exact top-min(k, n) leave as 64-bit candidates
+//     k-th best; every 4 tiles, if the buffer is nearly full, an exact radix selection cuts it
+//     back to k and raises the bar.  At the end the chunk's exact top-min(k, n) leave as 64-bit candidates
 //     (score key << 32 | ~entry, so equal scores order the lower entry first).
 // Kernel 2 (one CTA per query): the exact top-k of the union of its chunks' candidates (the
 //   global top-k is contained in it), sorted by score descending then entry ascending.
@@ -42,16 +41,17 @@ using namespace tc;
 
 constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 8;
 constexpr int kChunk = 16384;                 // most keys per CTA
-constexpr int kCap = 4096;                    // candidate buffer (>= k + 2 tiles for k <= 2048)
-constexpr int kProdWarp = 0, kScaleWarp0 = 1, kEpiWarp0 = 5, kMmaWarp = 9;
+constexpr int kCap = 4096;                    // candidate buffer (> k + kCheck tiles for k <= 2048)
+constexpr int kCheck = 4;                     // tiles between checks of the buffer's fill
+constexpr int kProdWarp = 0, kEpiWarp0 = 1, kMmaWarp = 5;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kEpiBar = 1;                    // named barrier of the 4 epilogue warps
 constexpr uint32_t kTileCodes = kKT * kDI / 2; // 8192 B
 
 constexpr uint32_t OFF_ST = 0;                              // 8 x 8 KB codes (64-byte swizzle)
 constexpr uint32_t OFF_Q = OFF_ST + kStages * kTileCodes;    // query codes [64 x 64 B]
-constexpr uint32_t OFF_SCL = OFF_Q + 4096;                   // 8 x 128 scale words
-constexpr uint32_t OFF_W = OFF_SCL + kStages * 512;          // w [64] fp32
+constexpr uint32_t OFF_SCL = OFF_Q + 4096;                   // 8 x 128 scale words, then the query's
+constexpr uint32_t OFF_W = OFF_SCL + (kStages + 1) * 512;    // w [64] fp32
 constexpr uint32_t OFF_BUF = OFF_W + 256;                    // 2 x kCap candidates
 constexpr uint32_t OFF_SEL = OFF_BUF + 2 * kCap * 8;         // selection scratch (< 2 KB)
 constexpr uint32_t OFF_MISC = OFF_SEL + 2048;                // counters
@@ -61,14 +61,14 @@ constexpr uint32_t SMEM_USED = OFF_TMEM + 16;
 constexpr uint32_t SMEM_ALLOC = ((SMEM_USED + 127) / 128) * 128 + 1024;
 
 // TMEM columns: accumulators 64 per buffer at 0, 64, 128, 192; the scale words of stage s at
-// 256 + 4s; the query's at kColSfb.  Scale words sit in the layout the 32x128b.warpx4 copy produces: in every
-// lane quadrant, lane l of column c + j holds the word of row l + 32j.
+// 256 + 4s; the query's at kColSfb.  The 32x128b.warpx4 copy puts them in every lane quadrant:
+// lane l of column c + j holds the word of row l + 32j.
 constexpr int kDBufs = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t kColSfa = 64 * kDBufs, kColSfb = kColSfa + 4 * kStages;
 
-enum { B_FULL = 0, B_SFULL = B_FULL + kStages, B_EMPTY = B_SFULL + kStages, B_DFULL = B_EMPTY + kStages,
-       B_DEMPTY = B_DFULL + kDBufs, B_QFULL = B_DEMPTY + kDBufs, B_SFB, B_FINAL, NUM_BARS };
+enum { B_FULL = 0, B_EMPTY = B_FULL + kStages, B_DFULL = B_EMPTY + kStages, B_DEMPTY = B_DFULL + kDBufs,
+       B_QFULL = B_DEMPTY + kDBufs, B_FINAL, NUM_BARS };
 static_assert(NUM_BARS * 8 <= 512, "barrier space");
 static_assert(sizeof(SelectSmem<uint32_t>) <= 2048, "selection scratch");
 
@@ -96,13 +96,6 @@ __device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity)
 }
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync %0, 128;" ::"n"(kEpiBar) : "memory"); }
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
 
 // ------------------------------------------------------------------------------------------
 // kernel 1: FP4 key scan (tcgen05 kind::mxf4) + streaming chunk top-k
@@ -136,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
         for (int b = 0; b < NUM_BARS; ++b) {
             uint32_t cnt = 1;
             if (b >= B_FULL && b < B_FULL + kStages) cnt = 1 + 32; // expect_tx arrive + 32 cp.async arrivals
-            if ((b >= B_SFULL && b < B_SFULL + kStages) || b == B_SFB || (b >= B_DEMPTY && b < B_DEMPTY + kDBufs)) cnt = 4;
+            if (b >= B_DEMPTY && b < B_DEMPTY + kDBufs) cnt = 4;
             mbar_init(bar(b), cnt);
         }
         mbar_init_fence();
@@ -145,6 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
         misc[M_OUT] = 0;
     }
     if (tid < kHI) reinterpret_cast<float *>(sp + OFF_W)[tid] = a.w[r * kHI + tid];
+    if (tid < 128) { // the query's scale words in the copy layout (rows 64-127 zero)
+        const int l = tid & 31, j = tid >> 5, h = l + 32 * j;
+        reinterpret_cast<uint32_t *>(sp + OFF_SCL + kStages * 512)[4 * l + j] =
+            h < kHI ? reinterpret_cast<const uint32_t *>(a.q4.scales)[r * kHI + h] : 0u;
+    }
+    fence_proxy_async_smem();
     if (warp == kMmaWarp) tmem_alloc(base + OFF_TMEM, TMEM_COLS);
     tc_fence_before();
     __syncthreads();
@@ -164,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const int64_t row0 = key0 + (int64_t)i * kKT;
             const int valid = n - i * kKT < kKT ? n - i * kKT : kKT; // keys of the chunk in this tile
             for (int j = lane; j < valid; j += 32)
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + OFF_SCL + st * 512u + 4u * j),
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + OFF_SCL + st * 512u +
+                                                                          16u * (j & 31) + 4u * (j >> 5)),
                              "l"(scales + row0 + j)
                              : "memory");
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_FULL + st)) : "memory");
@@ -172,30 +172,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
                 mbar_arrive_expect_tx(bar(B_FULL + st), kTileCodes);
                 tma_load_2d(base + OFF_ST + st * kTileCodes, &maps.k, 0, (int32_t)row0, bar(B_FULL + st));
             }
-        }
-    } else if (warp >= kScaleWarp0 && warp < kEpiWarp0) {
-        const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        { // the query's scale words (64 rows; rows 64-127 of the layout unused)
-            const uint32_t *qs = reinterpret_cast<const uint32_t *>(a.q4.scales) + r * kHI;
-            tmem_st4(tq + kColSfb, qs[lane], qs[lane + 32], 0u, 0u);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SFB));
-        }
-        for (int i = 0; i < ntiles && ok; ++i) {
-            const uint32_t st = i % kStages;
-            if (!wwait(bar(B_FULL + st), (i / kStages) & 1)) { ok = false; break; }
-            const int valid = n - i * kKT;
-            const uint32_t sb = base + OFF_SCL + st * 512u;
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) w[j] = (lane + 32 * j < valid) ? lds32(sb + 4u * (lane + 32 * j)) : 0u;
-            tmem_st4(tq + kColSfa + 4u * st, w[0], w[1], w[2], w[3]);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SFULL + st));
         }
     } else if (warp >= kEpiWarp0 && warp < kMmaWarp) {
         const int quad = warp & 3, etid = tid - 32 * kEpiWarp0;
@@ -240,12 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             } else if (lane == 0) {
                 misc[M_ABORT] = 1;
             }
+            if ((i + 1) % kCheck != 0 && i + 1 != ntiles) continue; // the buffer has room for kCheck tiles
             epi_sync();
             const bool abort = misc[M_ABORT] != 0;
             const int cnt = misc[M_COUNT];
             epi_sync(); // every warp has read the count before any appends the next tile's keys
             if (abort) { ok = false; break; }
-            if (cnt > kCap - kKT && cnt > a.k) { // cut the buffer back to the k best, raise the bar
+            if (cnt > kCap - kCheck * kKT && cnt > a.k) { // cut the buffer back to the k best, raise the bar
                 theta = block_kth64<128, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
                 if (etid == 0) misc[M_OUT] = 0;
                 epi_sync();
@@ -279,16 +256,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             *out_count = 0;
         }
     } else if (warp == kMmaWarp && lane == 0) {
-        ok = mbar_wait(bar(B_QFULL), 0) && mbar_wait(bar(B_SFB), 0);
+        ok = mbar_wait(bar(B_QFULL), 0);
+        if (ok) {
+            tc_fence_after();
+            tmem_cp_32x128b_x4(tmem + kColSfb, sdesc_plain(base + OFF_SCL + kStages * 512u, 128, 128));
+        }
         for (int i = 0; i < ntiles && ok; ++i) {
             const uint32_t st = i % kStages, db = i % kDBufs;
-            if (!mbar_wait(bar(B_FULL + st), (i / kStages) & 1) || !mbar_wait(bar(B_SFULL + st), (i / kStages) & 1)) {
-                ok = false;
-                break;
-            }
+            if (!mbar_wait(bar(B_FULL + st), (i / kStages) & 1)) { ok = false; break; }
+            fence_proxy_async_smem(); // the cp.async scale words, read next by the tensor pipe
             if (i >= kDBufs && !mbar_wait(bar(B_DEMPTY + db), ((i / kDBufs) - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t a_tile = base + OFF_ST + st * kTileCodes;
+            tmem_cp_32x128b_x4(tmem + kColSfa + 4u * st, sdesc_plain(base + OFF_SCL + st * 512u, 128, 128));
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh) { // K = 0..63 (scale bytes 0-1), 64..127 (bytes 2-3)
                 mma_mxf4(tmem + db * 64u, sdesc_sw64(a_tile + 32u * kh, 512), sdesc_sw64(base + OFF_Q + 32u * kh, 512),

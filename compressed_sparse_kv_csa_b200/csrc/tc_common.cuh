@@ -93,6 +93,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
                  : "memory");
 }
 
+// TMA gather of 4 rows (y0..y3) x the box width at column x (2-D map with a one-row box) into
+// shared memory as a 4-row block; completes 4 x box bytes of the transaction count of `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int32_t x, int32_t y0, int32_t y1,
+                                            int32_t y2, int32_t y3, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+                 : "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // tcgen05
 // ------------------------------------------------------------------------------------------
@@ -208,6 +218,26 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
                  "setp.ne.b32 p, %6, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
                  "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate));
+}
+
+// Shared-memory descriptor without swizzle (core matrices of 8 rows x 16 bytes): LBO / SBO = byte
+// strides between core matrices along the leading / strided dimension.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// Copy 32 rows x 16 bytes of shared memory (descriptor) into 4 TMEM columns at `taddr`,
+// replicated into all four lane quadrants: lane l of column c + j receives bytes 4j..4j+3 of
+// row l.  Ordered with the MMAs issued later by the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
 }
 
 // 32 lanes x 4 consecutive 32-bit columns: thread i of the warp writes lane (base + i).

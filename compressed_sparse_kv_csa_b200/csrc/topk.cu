@@ -7,8 +7,8 @@
 //
 // One CTA per query row.  Radix select over order-preserving 32-bit keys of the fp32 scores
 // (8-bit digits over the bits that differ within the row, select.cuh) finds the exact k-th key; entries
-// above it are taken unordered, entries equal to it are taken in index order by a block-wide
-// ordered scan, and the k_eff winners are then sorted in shared memory (bitonic, 64-bit keys
+// above it are taken unordered, entries equal to it are collected and the lowest-index ones kept
+// (a second selection over the tie list), and the k_eff winners are then sorted in shared memory (bitonic, 64-bit keys
 // (score key, inverted index)).
 #include "common.cuh"
 #include "select.cuh"
@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
 {
     __shared__ unsigned long long sel[TK_MAX];
     __shared__ SelectSmem<uint32_t> ssel;
-    __shared__ int s_cnt, s_warp[TK_THREADS / 32], s_eq_taken;
+    __shared__ uint32_t ties[TK_MAX];
+    __shared__ int s_cnt, s_eq, s_warp[TK_THREADS / 32], s_eq_taken;
     extern __shared__ uint32_t skeys[]; // STAGED only
 
     const int64_t r = blockIdx.x;
@@ -64,38 +65,55 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     int n_gt = 0;       // number of keys strictly above thr
     if (nv > k) {
         block_kth<TK_THREADS, uint32_t>((int)nv, k, [&](int i) { return key(i); }, &ssel, thr, n_gt);
-        const int rem = k - n_gt;
-        if (tid == 0) { s_cnt = 0; s_eq_taken = 0; }
+        const int need = k - n_gt; // entries equal to the threshold that are taken: the lowest indices
+        if (tid == 0) { s_cnt = 0; s_eq = 0; s_eq_taken = 0; }
         __syncthreads();
-        // strictly greater: unordered append
+        // strictly greater: unordered append; equal: their indices into the tie list
         for (int64_t s = tid; s < nv; s += TK_THREADS) {
             const uint32_t kv = key(s);
             if (kv > thr) {
                 const int pos = atomicAdd(&s_cnt, 1);
                 if (pos < n_gt) sel[pos] = ((unsigned long long)kv << 32) | (0xffffffffu - (uint32_t)s);
+            } else if (kv == thr) {
+                const int e = atomicAdd(&s_eq, 1);
+                if (e < TK_MAX) ties[e] = (uint32_t)s;
             }
         }
         __syncthreads();
-        // equal to the threshold: the lowest indices first (ordered block scan)
-        const int need = rem;
-        for (int64_t base = 0; base < nv; base += TK_THREADS) {
-            if (s_eq_taken >= need) break; // uniform: read after a barrier
-            const int64_t s = base + tid;
-            const bool eq = (s < nv) && (key(s) == thr);
-            const unsigned bal = __ballot_sync(0xffffffffu, eq);
-            const int lane = tid & 31, wid = tid >> 5;
-            if (lane == 0) s_warp[wid] = __popc(bal);
-            __syncthreads();
-            int before = 0, total = 0;
-            for (int w = 0; w < TK_THREADS / 32; ++w) {
-                if (w < wid) before += s_warp[w];
-                total += s_warp[w];
+        const int n_eq = s_eq; // >= need
+        const unsigned long long hi = (unsigned long long)thr << 32;
+        if (n_eq <= TK_MAX) {
+            uint32_t lim = 0; // take the ties whose inverted index is >= lim
+            if (n_eq > need) {
+                int g;
+                block_kth<TK_THREADS, uint32_t>(n_eq, need, [&](int e) { return 0xffffffffu - ties[e]; }, &ssel, lim, g);
             }
-            const int rank = s_eq_taken + before + __popc(bal & ((1u << lane) - 1u));
-            if (eq && rank < need) sel[n_gt + rank] = ((unsigned long long)thr << 32) | (0xffffffffu - (uint32_t)s);
+            if (tid == 0) s_cnt = 0;
             __syncthreads();
-            if (tid == 0) s_eq_taken += total;
-            __syncthreads();
+            for (int e = tid; e < n_eq; e += TK_THREADS) {
+                const uint32_t inv = 0xffffffffu - ties[e];
+                if (inv >= lim) sel[n_gt + atomicAdd(&s_cnt, 1)] = hi | inv;
+            }
+        } else { // more ties than the list holds: ordered block scan from the lowest index
+            for (int64_t base = 0; base < nv; base += TK_THREADS) {
+                if (s_eq_taken >= need) break; // uniform: read after a barrier
+                const int64_t s = base + tid;
+                const bool eq = (s < nv) && (key(s) == thr);
+                const unsigned bal = __ballot_sync(0xffffffffu, eq);
+                const int lane = tid & 31, wid = tid >> 5;
+                if (lane == 0) s_warp[wid] = __popc(bal);
+                __syncthreads();
+                int before = 0, total = 0;
+                for (int w = 0; w < TK_THREADS / 32; ++w) {
+                    if (w < wid) before += s_warp[w];
+                    total += s_warp[w];
+                }
+                const int rank = s_eq_taken + before + __popc(bal & ((1u << lane) - 1u));
+                if (eq && rank < need) sel[n_gt + rank] = hi | (0xffffffffu - (uint32_t)s);
+                __syncthreads();
+                if (tid == 0) s_eq_taken += total;
+                __syncthreads();
+            }
         }
     } else {
         for (int64_t s = tid; s < nv; s += TK_THREADS)
