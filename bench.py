@@ -543,6 +543,67 @@ class OracleDecode:
                 f"hybrid attention over the selected rows + window {self.w.W}")
 
 
+class OracleMixed:
+    """The oracle on a bounded sample of the stacked decode: n_seq sequences spread evenly over
+    the batch's length order (shortest to longest) through the four layers, glue included.  Inputs are drawn and
+    dequantised once (untimed); run() times the oracle's indexer, top-k, attention and glue."""
+
+    def __init__(self, w, n_seq: int = 2, seed_rank: int = 0):
+        import oracle as O
+        self.w = w
+        H, c, Hi, di, W = w.H, w.c, w.H_I, w.d_I, w.W
+        lens = WL.mixed_lengths(w)
+        seqs = rank_sequences(w.B, seed_rank)
+        order = np.argsort(lens)[np.linspace(0, w.B - 1, n_seq).astype(np.int64)]
+        self.items = []
+        kinds = w.extra["layers"]
+        for b in order:
+            s, t = seqs[int(b)], int(lens[int(b)])
+            layers = []
+            for l, kind in enumerate(kinds):
+                m = w.extra["m_csa"] if kind == "csa" else w.extra["m_hca"]
+                nv = (t + 1) // m
+                L = {"csa": kind == "csa", "m": m, "nv": nv,
+                     "KV": O.dequant_kv(*O.quant_kv(WL.draw(w, "KV", 0, nv, layer=l, seq=s))),
+                     "win": O.dequant_kv(*O.quant_kv(WL.draw(w, "WIN", 0, W, layer=l, seq=s))),
+                     "sink": WL.draw(w, "sink", 0, 1, layer=l, seq=seed_rank)[0]}
+                if L["csa"]:
+                    L["Kd"] = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "KI", 0, nv, layer=l, seq=s)))
+                    L["w"] = WL.draw(w, "w", 0, 1, layer=l, seq=s)
+                if l + 1 < len(kinds):
+                    L["P"] = WL.draw(w, "P", 0, c, layer=l)
+                    L["Rm"] = WL.draw(w, "Rm", 0, di, layer=l)
+                layers.append(L)
+            q0 = WL.draw(w, "q", 0, 1, layer=0, seq=s).reshape(1, H, c).astype(np.float64)
+            self.items.append((t, q0, layers))
+        self.n = n_seq
+
+    def run(self):
+        import oracle as O
+        w = self.w
+        H, c, Hi, di, W = w.H, w.c, w.H_I, w.d_I, w.W
+        t0 = time.perf_counter()
+        for t, q, layers in self.items:
+            zi = None
+            for l, L in enumerate(layers):
+                if L["csa"]:
+                    Qd = O.dequant_fp4(*O.quant_fp4(zi.astype(np.float32))).reshape(1, Hi, di)
+                    idx, _ = O.indexer_topk(Qd, L["w"], L["Kd"], np.array([t]), L["m"], w.k)
+                    o, _ = O.hybrid_attn_decode(q, L["KV"], [0], [t], L["win"], [W], L["sink"], 1.0, L["m"], W, idx=idx)
+                else:
+                    o, _ = O.hybrid_attn_decode(q, L["KV"], [0], [t], L["win"], [W], L["sink"], 1.0, L["m"], W)
+                if l + 1 < len(layers):
+                    ob = O.bf16_value(O.bf16_bits(o.reshape(H, c)))
+                    qn, zi = O.decode_glue(ob, L["P"], L["Rm"])
+                    q = O.bf16_value(O.bf16_bits(qn)).reshape(1, H, c).astype(np.float64)
+        secs = time.perf_counter() - t0
+        return self.n / secs, secs
+
+    def describe(self):
+        return (f"{self.n} of the {self.w.B} sequences, evenly spaced in length order, through the "
+                f"{len(self.w.extra['layers'])}-layer stack (indexer, top-k, attention, glue)")
+
+
 def oracle_hca_sample(w, target_s: float = 10.0):
     """cpu_baseline leg: calibrate the sample so the oracle's attention work takes ~target_s."""
     probe = OracleHca(w, 16)
@@ -683,12 +744,13 @@ def main():
             "clocks": clk.summary(),
             "gpu_launches": job.launches_per_step * args.steps,
         }
-        if not args.no_cpu_baseline and world == 1 and args.workload in ("hca_prefill_32k", "csa_decode_1m"):
+        if not args.no_cpu_baseline and world == 1 and args.workload in ("hca_prefill_32k", "csa_decode_1m",
+                                                                          "mixed_decode_64"):
             import oracle as O
             if args.workload == "hca_prefill_32k":
                 tps, secs, desc = oracle_hca_sample(w)
             else:
-                job_o = OracleDecode(w, 4)
+                job_o = OracleDecode(w, 4) if args.workload == "csa_decode_1m" else OracleMixed(w, 8)
                 tps, secs = job_o.run()
                 desc = job_o.describe()
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
@@ -704,7 +766,12 @@ def reference_arm(args, w, world, rank):
     if rank != 0:
         return
     import oracle as O
-    job = OracleDecode(w, 1) if w.kind == "csa_decode" else OracleHca(w, 256)
+    if w.kind == "csa_decode":
+        job = OracleDecode(w, 1)
+    elif w.kind == "mixed_decode":
+        job = OracleMixed(w, 2)
+    else:
+        job = OracleHca(w, 256)
     desc = job.describe()
     for _ in range(max(args.warmup, 3)):
         job.run()
