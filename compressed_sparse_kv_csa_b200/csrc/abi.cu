@@ -298,8 +298,15 @@ int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *co
     const int64_t max_keys = (int64_t)W + (idx ? k : max_nvis);
     uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + kAlign - 1) / kAlign * kAlign;
     a.part = reinterpret_cast<float *>(base);
-    a.n_chunks = decode_tc_chunks(max_keys);
-    a.chunk = 128;
+    // tensor-core path: items of tpc 128-key tiles, about four items per SM over the whole batch
+    // (estimated from the longest key list); one tile per item when the batch is small
+    {
+        const int64_t tiles = decode_tc_chunks(max_keys);
+        int64_t tpc = (int64_t)B * tiles / (4 * 148);
+        tpc = tpc < 1 ? 1 : (tpc > 8 ? 8 : tpc);
+        a.chunk = (int)(128 * tpc);
+        a.n_chunks = (int)((tiles + tpc - 1) / tpc);
+    }
     if (decode_attn_tc_eligible(a)) { // 64 heads x 512 channels: tcgen05 split-K + merge
         cudaError_t e = launch_attn_decode_tc(a, S(stream));
         if (e != cudaSuccess) return CSA_ERR_CUDA;

@@ -7,17 +7,19 @@
 // concatenated); KV cache with BF16 RoPE dims and FP8 for the rest ("Mind Observatory: Uncovering
 // the technical ledger of DeepSeek-V4"); the per-head sink is folded in by the merge kernel.
 //
-// Work items = (sequence, chunk of 128 keys of its key list); persistent CTAs (one per SM) walk
-// the items, so the many empty chunks of short sequences in a mixed batch cost no launch.  For each
-// non-empty item a CTA:
-//   1. stages q [64 x 512] (bf16) and gathers its 128 key rows -- window rows first, then the
-//      top-k (CSA) or visible (HCA) compressed rows -- dequantising the FP8 part (code x row scale)
-//      to bf16 next to the BF16 RoPE part, all in 128-byte-swizzled shared memory;
+// Work items = (sequence, chunk of `chunk` keys = 1-8 tiles of 128 of its key list); persistent
+// CTAs (one per SM) walk the items, so the many empty chunks of short sequences in a mixed batch
+// cost no launch.  For each non-empty item a CTA stages q [64 x 512] (bf16) once, then for each
+// 128-key tile of the item:
+//   1. gathers its key rows -- window rows first, then the top-k (CSA) or visible (HCA)
+//      compressed rows -- dequantising the FP8 part (code x row scale) to bf16 next to the BF16
+//      RoPE part, in 128-byte-swizzled shared memory;
 //   2. one thread issues S = Q K^T (tcgen05 M=64, N=128, K=512) into TMEM;
-//   3. 4 warps take the softmax of their 16 heads over the chunk (lanes l and l+16 split the
-//      keys), writing P (bf16) to shared memory and (max, sum) to the workspace;
-//   4. O = P V (two M=64 x N=256 x K=128 MMAs, V = the same tile read MN-major) into TMEM, and
-//      the unnormalised O rows go to the workspace for the split-K merge.
+//   3. 4 warps take the online softmax of their 16 heads (lanes l and l+16 split the keys; the
+//      running max moves, and O is rescaled in TMEM, only when a tile raises it by more than 8),
+//      writing P (bf16) to shared memory;
+//   4. O (+)= P V (two M=64 x N=256 x K=128 MMAs, V = the same tile read MN-major) in TMEM.
+// The item's (max, sum, unnormalised O) rows go to the workspace for the split-K merge.
 #include "common.cuh"
 #include "tc_common.cuh"
 
@@ -125,8 +127,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
     }
     __syncthreads();
     const int64_t n_items = (int64_t)a.B * a.n_chunks;
-    uint32_t ph = 0; // parity of bar_s / bar_o for the next non-empty item
+    const int tpc = a.chunk / kKT; // 128-key tiles per item
+    uint32_t ph = 0;               // parity of bar_s / bar_o for the next tile
     bool ok = true;
+    int64_t *rows = reinterpret_cast<int64_t *>(sp + OFF_ROWS);
+    const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
+    const bool upper = lane < 16;
+    const int row = 16 * (warp & 3) + (lane & 15); // head of this softmax lane (warps 0-3)
+    const float sl2 = a.scale * kLog2e;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const int b = (int)(item / a.n_chunks), chunk = (int)(item % a.n_chunks);
         int n_win;
@@ -137,44 +145,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
         } else {
             seq_counts(b, n_win, n_keys);
         }
-        const int64_t j0 = (int64_t)chunk * kKT;
+        const int64_t t_beg = (int64_t)chunk * tpc, n_tiles = (n_keys + kKT - 1) / kKT;
+        const int64_t t_end = t_beg + tpc < n_tiles ? t_beg + tpc : n_tiles;
         float *part = a.part + ((int64_t)b * a.n_chunks + chunk) * kH * (kC + 2);
-        if (j0 >= n_keys) { // empty chunk: a neutral partial (CTA-uniform)
+        if (t_beg >= t_end) { // empty chunk: a neutral partial (CTA-uniform)
             for (int h = tid; h < kH; h += kThreads) {
                 part[(int64_t)h * (kC + 2)] = -INFINITY;
                 part[(int64_t)h * (kC + 2) + 1] = 0.f;
             }
             continue;
         }
-
-        // ---- resolve the chunk's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
-        int64_t *rows = reinterpret_cast<int64_t *>(sp + OFF_ROWS);
-        if (tid < kKT) {
-            const int64_t j = j0 + tid;
-            int64_t code = -1;
-            if (j < n_keys && j < n_win) {
-                code = (int64_t)b * a.W + j;
-            } else if (j < n_keys) {
-                const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
-                if (s >= 0) {
-                    const int64_t r = a.comp_off[b] + s;
-                    if (r >= 0 && r < a.comp.n) code = r | (1ll << 62);
-                    else flag_error(a.err, CSA_DEVERR_INDEX);
-                }
-            }
-            rows[tid] = code;
-            valid[tid] = code >= 0 ? 1 : 0;
-        }
         // ---- stage q (all threads): 16 independent 16-byte loads per thread in flight
         for (int e0 = tid; e0 < kH * (kC / 8); e0 += 16 * kThreads) {
             uint4 v[16];
-    #pragma unroll
+#pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int e = e0 + u * kThreads;
                 if (e < kH * (kC / 8))
                     v[u] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * kH + (e >> 6)) * kC + 8 * (e & 63)));
             }
-    #pragma unroll
+#pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int e = e0 + u * kThreads;
                 if (e < kH * (kC / 8)) {
@@ -183,146 +173,185 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
                 }
             }
         }
-        __syncthreads();
-        // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as is;
-        // 12 independent loads per thread in flight
-        const int cn = kC - a.comp.rope_dims; // FP8 channels (448), RoPE channels after them
-        constexpr int kU = 12;
-        for (int e0 = tid; e0 < kKT * (kC / 8); e0 += kU * kThreads) {
-            uint4 raw[kU];
-            float sc[kU];
-            int kind[kU]; // 0 empty, 1 FP8, 2 RoPE
-    #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int e = e0 + u * kThreads;
-                kind[u] = 0;
-                raw[u] = make_uint4(0, 0, 0, 0);
-                sc[u] = 0.f;
-                if (e < kKT * (kC / 8)) {
-                    const int64_t code = rows[e >> 6];
-                    if (code >= 0) {
-                        const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
-                        const int64_t row = code & ((1ll << 62) - 1);
-                        const int ch = 8 * (e & 63);
-                        if (ch < cn) {
-                            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(kv.fp8 + row * cn + ch));
-                            raw[u].x = c.x;
-                            raw[u].y = c.y;
-                            sc[u] = __ldg(kv.scale + row);
-                            kind[u] = 1;
-                        } else {
-                            raw[u] = __ldg(reinterpret_cast<const uint4 *>(kv.rope + row * kv.rope_dims + (ch - cn)));
-                            kind[u] = 2;
+        float m_run = -INFINITY, l_run = 0.f; // online softmax of this lane's row (log2 domain)
+        for (int64_t tile = t_beg; tile < t_end && ok; ++tile) {
+            const bool first = tile == t_beg;
+            const int64_t j0 = tile * kKT;
+            // ---- resolve the tile's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
+            if (tid < kKT) {
+                const int64_t j = j0 + tid;
+                int64_t code = -1;
+                if (j < n_keys && j < n_win) {
+                    code = (int64_t)b * a.W + j;
+                } else if (j < n_keys) {
+                    const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
+                    if (s >= 0) {
+                        const int64_t r = a.comp_off[b] + s;
+                        if (r >= 0 && r < a.comp.n) code = r | (1ll << 62);
+                        else flag_error(a.err, CSA_DEVERR_INDEX);
+                    }
+                }
+                rows[tid] = code;
+                valid[tid] = code >= 0 ? 1 : 0;
+            }
+            __syncthreads();
+            // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as
+            // is; 12 independent loads per thread in flight
+            constexpr int kU = 12;
+            for (int e0 = tid; e0 < kKT * (kC / 8); e0 += kU * kThreads) {
+                uint4 raw[kU];
+                float sc[kU];
+                int kind[kU]; // 0 empty, 1 FP8, 2 RoPE
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int e = e0 + u * kThreads;
+                    kind[u] = 0;
+                    raw[u] = make_uint4(0, 0, 0, 0);
+                    sc[u] = 0.f;
+                    if (e < kKT * (kC / 8)) {
+                        const int64_t code = rows[e >> 6];
+                        if (code >= 0) {
+                            const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
+                            const int64_t rw = code & ((1ll << 62) - 1);
+                            const int ch = 8 * (e & 63);
+                            if (ch < cn) {
+                                const uint2 c = __ldg(reinterpret_cast<const uint2 *>(kv.fp8 + rw * cn + ch));
+                                raw[u].x = c.x;
+                                raw[u].y = c.y;
+                                sc[u] = __ldg(kv.scale + rw);
+                                kind[u] = 1;
+                            } else {
+                                raw[u] = __ldg(reinterpret_cast<const uint4 *>(kv.rope + rw * kv.rope_dims + (ch - cn)));
+                                kind[u] = 2;
+                            }
                         }
                     }
                 }
-            }
-    #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int e = e0 + u * kThreads;
-                if (e < kKT * (kC / 8)) {
-                    const int jj = e >> 6, cc = e & 63;
-                    const uint4 v = kind[u] == 1 ? fp8x8_to_bf16(make_uint2(raw[u].x, raw[u].y), sc[u]) : raw[u];
-                    sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        if (warp == kMmaWarp && lane == 0) { // S = Q K^T
-    #pragma unroll
-            for (int s = 0; s < 8; ++s)
-    #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + kColS, sdesc_sw128(sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024),
-                             sdesc_sw128(sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024), IDESC_S, (s | kk) != 0);
-            mma_commit(bar_s);
-        }
-        const bool upper = lane < 16;
-        const int row = 16 * (warp & 3) + (lane & 15);
-        if (warp < 4) { // softmax of the chunk: lane l keys 0-63, lane l+16 keys 64-127 of head `row`
-            const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_s, ph));
-            if (ok) {
-                tc_fence_after();
-                uint32_t r0[32], r1[32], r2[32], r3[32];
-                tmem_ld32(tw + kColS, r0);
-                tmem_ld32(tw + kColS + 32, r1);
-                tmem_ld32(tw + kColS + 64, r2);
-                tmem_ld32(tw + kColS + 96, r3);
-                tmem_ld_wait();
-                float sv[64];
-                const int kb = upper ? 0 : 64;
-                const float sl2 = a.scale * kLog2e;
-                float mt = -INFINITY;
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
-                    const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
-                    float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
-                    s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
-                    s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
-                    sv[e] = s0;
-                    sv[32 + e] = s1;
-                    mt = fmaxf(mt, fmaxf(s0, s1));
-                }
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                float ls = 0.f;
-    #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const float p = (mt == -INFINITY) ? 0.f : ex2(sv[e] - mt);
-                    sv[e] = p;
-                    ls += p;
-                }
-                ls += __shfl_xor_sync(0xffffffffu, ls, 16);
-                const uint32_t psub = sP + (uint32_t)(kb >> 6) * 8192u;
-    #pragma unroll
-                for (int g = 0; g < 8; ++g)
-                    sts4(psub + sw128_off(row, 8 * g),
-                         make_uint4(pk_bf16(sv[8 * g], sv[8 * g + 1]), pk_bf16(sv[8 * g + 2], sv[8 * g + 3]),
-                                    pk_bf16(sv[8 * g + 4], sv[8 * g + 5]), pk_bf16(sv[8 * g + 6], sv[8 * g + 7])));
-                if (upper) {
-                    part[(int64_t)row * (kC + 2)] = (mt == -INFINITY) ? -INFINITY : mt * kLn2; // natural-log max
-                    part[(int64_t)row * (kC + 2) + 1] = ls;
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int e = e0 + u * kThreads;
+                    if (e < kKT * (kC / 8)) {
+                        const int jj = e >> 6, cc = e & 63;
+                        const uint4 v = kind[u] == 1 ? fp8x8_to_bf16(make_uint2(raw[u].x, raw[u].y), sc[u]) : raw[u];
+                        sts4(sK + (uint32_t)(cc >> 3) * 16384u + sw128_off(jj, (cc & 7) * 8), v);
+                    }
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-        }
-        __syncthreads();
-        ok = __syncthreads_and(ok);
-        if (warp == kMmaWarp && lane == 0 && ok) { // O = P V
+            __syncthreads();
             tc_fence_after();
-    #pragma unroll
-            for (int h = 0; h < 2; ++h)
-    #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(h ? tmem : tmem + TMEM_O,
-                             sdesc_sw128(sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024),
-                             sdesc_sw128(sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024), IDESC_PV, kk > 0);
-            mma_commit(bar_o);
-        }
-        if (warp < 4 && ok) { // unnormalised O rows -> workspace (lane l: channels 256-511, l+16: 0-255)
-            const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-            if (__all_sync(0xffffffffu, mbar_wait(bar_o, ph))) {
-                tc_fence_after();
-                float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tw + 32u * c, r);
+
+            if (warp == kMmaWarp && lane == 0) { // S = Q K^T
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + kColS, sdesc_sw128(sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024),
+                                 sdesc_sw128(sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024), IDESC_S, (s | kk) != 0);
+                mma_commit(bar_s);
+            }
+            if (warp < 4) { // softmax of the tile: lane l keys 0-63, lane l+16 keys 64-127 of head `row`
+                const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_s, ph));
+                if (ok) {
+                    tc_fence_after();
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(tw + kColS, r0);
+                    tmem_ld32(tw + kColS + 32, r1);
+                    tmem_ld32(tw + kColS + 64, r2);
+                    tmem_ld32(tw + kColS + 96, r3);
                     tmem_ld_wait();
-                    // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
-                    // 8-byte stores are the widest that are aligned for every row
-    #pragma unroll
-                    for (int g = 0; g < 16; ++g)
-                        *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
-                            make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
+                    float sv[64];
+                    const int kb = upper ? 0 : 64;
+                    float mt = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
+                        const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
+                        float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
+                        s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
+                        s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
+                        sv[e] = s0;
+                        sv[32 + e] = s1;
+                        mt = fmaxf(mt, fmaxf(s0, s1));
+                    }
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                    // lazy rescale: the running max moves only when this tile raises it by more than 8
+                    const float m_new = fmaxf(m_run, mt);
+                    float resc = 1.f, m_use = m_run;
+                    if (m_new != -INFINITY && (m_run == -INFINITY || m_new > m_run + 8.f)) {
+                        resc = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+                        m_use = m_new;
+                    }
+                    float ls = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) {
+                        const float pv = (m_use == -INFINITY) ? 0.f : ex2(sv[e] - m_use);
+                        sv[e] = pv;
+                        ls += pv;
+                    }
+                    ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+                    l_run = l_run * resc + ls;
+                    m_run = m_use;
+                    // O of the earlier tiles (their P V is complete) moves to the new max
+                    if (!first && __any_sync(0xffffffffu, resc != 1.f)) {
+                        for (int c = 0; c < 8; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(tw + 32u * c, r);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * resc);
+                            tmem_st32(tw + 32u * c, r);
+                        }
+                        tmem_st_wait();
+                    }
+                    const uint32_t psub = sP + (uint32_t)(kb >> 6) * 8192u;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        sts4(psub + sw128_off(row, 8 * g),
+                             make_uint4(pk_bf16(sv[8 * g], sv[8 * g + 1]), pk_bf16(sv[8 * g + 2], sv[8 * g + 3]),
+                                        pk_bf16(sv[8 * g + 4], sv[8 * g + 5]), pk_bf16(sv[8 * g + 6], sv[8 * g + 7])));
                 }
-            } else {
-                ok = false;
+                fence_proxy_async_smem();
+                tc_fence_before();
+            }
+            ok = __syncthreads_and(ok);
+            if (warp == kMmaWarp && lane == 0 && ok) { // O (+)= P V
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(h ? tmem : tmem + TMEM_O,
+                                 sdesc_sw128(sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024),
+                                 sdesc_sw128(sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024), IDESC_PV,
+                                 (!first || kk > 0) ? 1u : 0u);
+                mma_commit(bar_o);
+            }
+            // the next tile's gather overwrites the keys (= values) and P: wait for P V everywhere
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o, ph));
+            tc_fence_after();
+            ok = __syncthreads_and(ok);
+            ph ^= 1;
+        }
+        if (warp < 4 && ok) { // (max, sum, unnormalised O) -> workspace (lane l: channels 256-511, l+16: 0-255)
+            const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
+            if (upper) {
+                part[(int64_t)row * (kC + 2)] = (m_run == -INFINITY) ? -INFINITY : m_run * kLn2; // natural-log max
+                part[(int64_t)row * (kC + 2) + 1] = l_run;
+            }
+            float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tw + 32u * c, r);
+                tmem_ld_wait();
+                // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
+                // 8-byte stores are the widest that are aligned for every row
+#pragma unroll
+                for (int g = 0; g < 16; ++g)
+                    *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
+                        make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
             }
             tc_fence_before();
         }
@@ -330,7 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
         tc_fence_before();
         ok = __syncthreads_and(ok);
         tc_fence_after();
-        ph ^= 1;
     } // items
     if (!ok && tid == 0) flag_error(a.err, CSA_DEVERR_TIMEOUT);
     if (warp == kMmaWarp && lane == 0) {

@@ -18,7 +18,8 @@
 //     reads (row l holds the words of keys l, l+32, l+64, l+96);
 //   * MMA lane: copies the tile's scale words into TMEM (tcgen05.cp 32x128b.warpx4), then two
 //     M=128 (keys) x N=64 (heads) x K=64 block-scaled MMAs into one of four TMEM accumulators;
-//   * 4 epilogue warps (one key per lane): score = w . ReLU(row of 64 head dot products), then a
+//   * 8 epilogue warps in two groups taking alternate tiles (one key per lane, a warp per TMEM
+//     lane quadrant): score = w . ReLU(row of 64 head dot products), then a
 //     streaming filter: a key enters the chunk's candidate buffer only if it beats the current
 //     k-th best; every 4 tiles, if the buffer is nearly full, an exact radix selection cuts it
 //     back to k and raises the bar.  At the end the chunk's exact top-min(k, n) leave as 64-bit candidates
@@ -43,9 +44,10 @@ constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 8;
 constexpr int kChunk = 16384;                 // most keys per CTA
 constexpr int kCap = 4096;                    // candidate buffer (> k + kCheck tiles for k <= 2048)
 constexpr int kCheck = 4;                     // tiles between checks of the buffer's fill
-constexpr int kProdWarp = 0, kEpiWarp0 = 1, kMmaWarp = 5;
+constexpr int kProdWarp = 0, kEpiWarp0 = 1, kEpiWarps = 8, kMmaWarp = kEpiWarp0 + kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kEpiBar = 1;                    // named barrier of the 4 epilogue warps
+constexpr int kEpiBar = 1;                    // named barrier of the 8 epilogue warps
 constexpr uint32_t kTileCodes = kKT * kDI / 2; // 8192 B
 
 constexpr uint32_t OFF_ST = 0;                              // 8 x 8 KB codes (64-byte swizzle)
@@ -95,7 +97,7 @@ __device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity)
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync %0, 128;" ::"n"(kEpiBar) : "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kEpiBar), "n"(kEpiThreads) : "memory"); }
 
 // ------------------------------------------------------------------------------------------
 // kernel 1: FP4 key scan (tcgen05 kind::mxf4) + streaming chunk top-k
@@ -174,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             }
         }
     } else if (warp >= kEpiWarp0 && warp < kMmaWarp) {
-        const int quad = warp & 3, etid = tid - 32 * kEpiWarp0;
+        const int quad = warp & 3, etid = tid - 32 * kEpiWarp0, grp = (warp - kEpiWarp0) >> 2;
         float w[kHI];
 #pragma unroll
         for (int h = 0; h < kHI; ++h) w[h] = reinterpret_cast<const float *>(sp + OFF_W)[h];
@@ -182,10 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
         unsigned long long *alt = buf + kCap;
         SelectSmem<uint32_t> *sel = reinterpret_cast<SelectSmem<uint32_t> *>(sp + OFF_SEL);
         unsigned long long theta = 0; // a key enters the buffer only above this
-        for (int i = 0; i < ntiles; ++i) {
+        const int npairs = (ntiles + 1) / 2;
+        for (int p = 0; p < npairs; ++p) { // group g takes tile 2p + g; both groups pass the same barriers
+            const int i = 2 * p + grp;
             const uint32_t db = i % kDBufs;
-            const bool got = wwait(bar(B_DFULL + db), (i / kDBufs) & 1);
-            if (got) {
+            const bool got = i >= ntiles || wwait(bar(B_DFULL + db), (i / kDBufs) & 1);
+            if (i >= ntiles) {
+            } else if (got) {
                 tc_fence_after();
                 uint32_t r0[32], r1[32];
                 const uint32_t ta = tmem + db * 64u + ((uint32_t)(32 * quad) << 16);
@@ -216,22 +221,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             } else if (lane == 0) {
                 misc[M_ABORT] = 1;
             }
-            if ((i + 1) % kCheck != 0 && i + 1 != ntiles) continue; // the buffer has room for kCheck tiles
+            if ((p + 1) % (kCheck / 2) != 0 && p + 1 != npairs) continue; // the buffer has room for kCheck tiles
             epi_sync();
             const bool abort = misc[M_ABORT] != 0;
             const int cnt = misc[M_COUNT];
             epi_sync(); // every warp has read the count before any appends the next tile's keys
             if (abort) { ok = false; break; }
             if (cnt > kCap - kCheck * kKT && cnt > a.k) { // cut the buffer back to the k best, raise the bar
-                theta = block_kth64<128, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
+                theta = block_kth64<kEpiThreads, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
                 if (etid == 0) misc[M_OUT] = 0;
                 epi_sync();
-                for (int j = etid; j < cnt; j += 128) {
+                for (int j = etid; j < cnt; j += kEpiThreads) {
                     const unsigned long long v = buf[j];
                     if (v >= theta) alt[atomicAdd(&misc[M_OUT], 1)] = v;
                 }
                 epi_sync();
-                for (int j = etid; j < a.k; j += 128) buf[j] = alt[j];
+                for (int j = etid; j < a.k; j += kEpiThreads) buf[j] = alt[j];
                 if (etid == 0) misc[M_COUNT] = a.k;
                 epi_sync();
             }
@@ -240,16 +245,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const int cnt = misc[M_COUNT];
             if (cnt > a.k) {
                 const unsigned long long thr =
-                    block_kth64<128, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
+                    block_kth64<kEpiThreads, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
                 if (etid == 0) misc[M_OUT] = 0;
                 epi_sync();
-                for (int j = etid; j < cnt; j += 128) {
+                for (int j = etid; j < cnt; j += kEpiThreads) {
                     const unsigned long long v = buf[j];
                     if (v >= thr) out[atomicAdd(&misc[M_OUT], 1)] = v;
                 }
                 if (etid == 0) *out_count = a.k;
             } else {
-                for (int j = etid; j < cnt; j += 128) out[j] = buf[j];
+                for (int j = etid; j < cnt; j += kEpiThreads) out[j] = buf[j];
                 if (etid == 0) *out_count = cnt;
             }
         } else if (etid == 0) {
@@ -294,9 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
 // ------------------------------------------------------------------------------------------
 constexpr int kMergeThreads = 1024;
 
+constexpr int kPivCap = 4096; // candidates above the sampled pivot that the merge selects from
+
+// pivot: the union is first filtered by a pivot taken from every 16th candidate (the 1.5 k / 16-th
+// best sample, which lies below the k-th best of the union with high probability), so the exact
+// selection runs on about 1.5 k candidates; when the filter keeps fewer than k or more than
+// kPivCap, the selection runs on the whole union.
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs a, int n_slots,
                                                                      const unsigned long long *cand,
-                                                                     const int *cand_count)
+                                                                     const int *cand_count, int pivot)
 {
     extern __shared__ unsigned long long mv[];
     __shared__ SelectSmem<uint32_t> msel;
@@ -339,16 +350,49 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
     }
     __syncthreads();
     const int ke = total < k ? total : k;
-    unsigned long long *sel = mv + total; // ke winners
+    unsigned long long *buf = mv + total;                   // candidates above the pivot
+    unsigned long long *sel = buf + (pivot ? kPivCap : 0);  // ke winners
     if (total > k) {
-        const unsigned long long thr = block_kth64<kMergeThreads>(total, k, [&](int i) { return mv[i]; }, &msel);
-        if (tid == 0) s_cnt = 0;
-        __syncthreads();
-        for (int i = tid; i < total; i += kMergeThreads) {
-            const unsigned long long v = mv[i];
-            if (v >= thr) {
-                const int p = atomicAdd(&s_cnt, 1);
-                if (p < ke) sel[p] = v;
+        bool done = false;
+        const int ns = total >> 4, ks = (3 * k) >> 5;
+        if (pivot && ks >= 1 && ns >= 2 * ks) {
+            const unsigned long long piv =
+                block_kth64<kMergeThreads>(ns, ks, [&](int i) { return mv[16 * i]; }, &msel);
+            if (tid == 0) s_cnt = 0;
+            __syncthreads();
+            for (int i = tid; i < total; i += kMergeThreads) {
+                const unsigned long long v = mv[i];
+                if (v >= piv) {
+                    const int p = atomicAdd(&s_cnt, 1);
+                    if (p < kPivCap) buf[p] = v;
+                }
+            }
+            __syncthreads();
+            const int c = s_cnt;
+            if (c >= k && c <= kPivCap) { // the k best of the union are all above the pivot
+                const unsigned long long thr =
+                    block_kth64<kMergeThreads>(c, k, [&](int i) { return buf[i]; }, &msel);
+                __syncthreads();
+                if (tid == 0) s_cnt = 0;
+                __syncthreads();
+                for (int i = tid; i < c; i += kMergeThreads) {
+                    const unsigned long long v = buf[i];
+                    if (v >= thr) sel[atomicAdd(&s_cnt, 1)] = v;
+                }
+                done = true;
+            }
+            __syncthreads();
+        }
+        if (!done) {
+            const unsigned long long thr = block_kth64<kMergeThreads>(total, k, [&](int i) { return mv[i]; }, &msel);
+            if (tid == 0) s_cnt = 0;
+            __syncthreads();
+            for (int i = tid; i < total; i += kMergeThreads) {
+                const unsigned long long v = mv[i];
+                if (v >= thr) {
+                    const int p = atomicAdd(&s_cnt, 1);
+                    if (p < ke) sel[p] = v;
+                }
             }
         }
     } else {
@@ -444,10 +488,12 @@ cudaError_t launch_indexer_decode(const IndexerArgs &a, void *ws, cudaStream_t s
     if (e != cudaSuccess) return e;
     int n2 = 1;
     while (n2 < a.k) n2 <<= 1;
-    const size_t msm = (size_t)(slots * a.k + n2) * 8;
+    size_t msm = (size_t)(slots * a.k + n2) * 8;
+    const int pivot = msm + (size_t)kPivCap * 8 <= 220 * 1024 ? 1 : 0;
+    if (pivot) msm += (size_t)kPivCap * 8;
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msm);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<(unsigned)a.Nq, kMergeThreads, msm, st>>>(a, slots, cand, cnt);
+    decode_merge_kernel<<<(unsigned)a.Nq, kMergeThreads, msm, st>>>(a, slots, cand, cnt, pivot);
     return cudaGetLastError();
 }
 
