@@ -55,6 +55,7 @@ enum { B_QFULL = 0, B_QEMPTY, B_KVFULL0, B_KVFULL1, B_KVEMPTY0, B_KVEMPTY1, B_SF
        B_FINAL, NUM_BARS };
 
 constexpr uint32_t IDESC_S = idesc_bf16_f32(64, 128, false, false);
+constexpr uint32_t IDESC_S64 = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(64, 256, false, true);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 16u << 16; // lane offset of O[:, 0:256] (the lower lane half)
@@ -350,10 +351,14 @@ __device__ __forceinline__ bool mma_role(const PrefillArgs &a, const Smem &S, ui
 {
     uint32_t q_ph = 0, kf_ph[2] = {0, 0}, p_ph = 0;
     for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
-        const int nt = n_tiles(n_compressed(a, t));
+        const int64_t n_cmp = n_compressed(a, t);
+        const int nt = n_tiles(n_cmp);
         if (!mbar_wait(S.bar(B_QFULL), q_ph)) return false;
         q_ph ^= 1;
         for (int i = 0; i < nt; ++i) {
+            // a compressed tile with at most 64 slots in use (its valid slots come first): half the
+            // MMA work (N = 64 for S, 64 keys for P V); the softmax masks the other slots anyway
+            const bool half = i > 0 && n_cmp - (int64_t)(i - 1) * kKT <= 64;
             for (int s = 0; s < 8; ++s) {
                 if ((s & 3) == 0) { // each key half arrives separately
                     const int h = s >> 2;
@@ -365,7 +370,7 @@ __device__ __forceinline__ bool mma_role(const PrefillArgs &a, const Smem &S, ui
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = sdesc_sw128(S.sQ + (uint32_t)s * 8192u + 32u * kk, 16, 1024);
                     const uint64_t bd = sdesc_sw128(S.sK + (uint32_t)s * 16384u + 32u * kk, 16, 1024);
-                    mma_bf16(tmem + kColS, ad, bd, IDESC_S, (s | kk) != 0);
+                    mma_bf16(tmem + kColS, ad, bd, half ? IDESC_S64 : IDESC_S, (s | kk) != 0);
                 }
             }
             mma_commit(S.bar(B_SFULL));
@@ -374,8 +379,7 @@ __device__ __forceinline__ bool mma_role(const PrefillArgs &a, const Smem &S, ui
             p_ph ^= 1;
             tc_fence_after();
             for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < (half ? 4 : 8); ++kk) {
                     const uint64_t ad = sdesc_sw128(S.sP + (uint32_t)(kk >> 2) * 8192u + 32u * (kk & 3), 16, 1024);
                     const uint64_t bd = sdesc_sw128(S.sK + (uint32_t)h * 65536u + 2048u * kk, 16384, 1024);
                     mma_bf16(h ? tmem : tmem + TMEM_O, ad, bd, IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);

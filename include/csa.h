@@ -205,7 +205,8 @@ int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t
  *   o[t,h,:] = sum e^z key / (e^{sink[h]} + sum e^z),  lse[t,h] = ln(e^{sink[h]} + sum e^z).
  *
  *   q [T, H, c], x_win [T, c], kv_comp [n_comp, c] in `dtype` (CSA_F32 / CSA_BF16)
- *   idx [T, k] int32 or NULL; entries outside [0, n_comp) are skipped (CSA_DEVERR_INDEX)
+ *   idx [T, k] int32 or NULL; negative entries (padding) are skipped, entries >= n_comp are
+ *            skipped and set CSA_DEVERR_INDEX
  *   sink [H] fp32 (-inf allowed: no sink);  o [T, H, c] in `dtype`;  lse [T, H] fp32 or NULL
  * Limits: c a multiple of 32 and <= 512, 1 <= H <= 128, 1 <= W <= 1024, k <= 4096.
  */
