@@ -379,6 +379,41 @@ def test_decode_attention_mixed_cache(C, use_idx):
     np.testing.assert_allclose(host(lse), lse_ref, atol=1e-2)
 
 
+def test_decode_attention_multi_tile_items(C):
+    """A batch large enough that the tensor-core decode takes several 128-key tiles per work item
+    (64 sequences, all visible entries, up to 6,000 of them): the online softmax across a chunk's
+    tiles, its lazy rescale, partial last items and sequences with a single short item."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, H, c, W, m = 64, 64, 512, 128, 4
+    g = np.random.default_rng(21)
+    nv = g.integers(50, 3000, size=Bn).astype(np.int64)
+    nv[7] = 6000
+    pos = nv * m + g.integers(0, m, size=Bn)
+    off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+    comp = WL.draw(w, "KV", 0, int(nv.sum()), seq=200)   # sequence b's entries: rows off[b] ...
+    win_len = np.full(Bn, W, np.int32)
+    win_len[3] = 17
+    win = WL.draw(w, "WIN", 0, Bn * W, seq=200)
+    q = WL.draw(w, "q", 0, Bn, seq=200).reshape(Bn, H, c)
+    sink = WL.draw(w, "sink", 0, 1)[0]
+    cf, cr, cs = O.quant_kv(comp)
+    wf, wr, ws = O.quant_kv(win)
+    o_ref, lse_ref = O.hybrid_attn_decode(WL.on_grid(q, "bf16"), O.dequant_kv(cf, cr, cs), off, pos,
+                                          O.dequant_kv(wf, wr, ws), win_len, sink, 1.0, m, W)
+    ckv = C.KvRows.empty(len(comp), c, 64, "cuda")
+    wkv = C.KvRows.empty(Bn * W, c, 64, "cuda")
+    C.csa_quantize_kv(dev(comp), ckv)
+    C.csa_quantize_kv(dev(win), wkv)
+    lse = torch.empty((Bn, H), dtype=torch.float32, device="cuda")
+    o = C.hybrid_attn_decode(dev(WL.on_grid(q, "bf16"), "bf16"), ckv, torch.from_numpy(off).cuda(),
+                             torch.from_numpy(pos).cuda(), wkv, dev_i(win_len), dev(sink), 1.0, m, W,
+                             max_nvis=int(nv.max()), lse=lse)
+    torch.cuda.synchronize()
+    assert C.csa_device_error() == 0
+    assert row_rel_err(host(o), o_ref).max() < 2e-2
+    np.testing.assert_allclose(host(lse), lse_ref, atol=1e-2)
+
+
 # ---------------------------------------------------------------------------------------------
 # the tiny CSA layer end to end (compress -> indexer -> top-k -> attention)
 # ---------------------------------------------------------------------------------------------
