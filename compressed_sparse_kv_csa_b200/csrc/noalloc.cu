@@ -54,6 +54,9 @@ int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t
                         int32_t *idx_out, float *score_out, void *stream)
 {
     if (Nq < 0 || max_nvis < 0) return CSA_ERR_INVALID_ARG;
+    if (Nq == 0) // nothing to score: the arguments are still checked, no device is needed
+        return indexer_topk(q, w, keys, fmt, q_pos, key_off, n_keys, Nq, H_I, d_I, m, k, max_nvis,
+                            idx_out, score_out, nullptr, 0, stream);
     const size_t need = indexer_topk_workspace_size(Nq, max_nvis, k);
     if (need > kStaticBytes) return CSA_ERR_SCRATCH_CAPACITY;
     cudaError_t err = cudaSuccess;

@@ -27,6 +27,8 @@
  *     launch failed (the CUDA error is left for cudaGetLastError()).  Kernels never trap: a
  *     bounded wait that runs out, or an index the kernel refuses to follow, sets a device error
  *     word that csa_device_error() reads back.
+ *   - A call with nothing to compute (no complete block, no rows, no queries, no tokens, no
+ *     sequences) runs its argument checks and returns CSA_OK without touching the device.
  *   - dtype codes: CSA_F32 (fp32) and CSA_BF16 (bf16, stored as uint16 bit patterns).
  *   - Numerics: inputs bf16 / fp32 / fp8 / fp4, all accumulation and softmax in fp32.
  */
@@ -177,7 +179,8 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
  * scratch is a file-scope device array of indexer_topk_static_capacity() = 4,194,304 fp32 scores
  * (16 MiB), which every GPU that loads this library holds until the process exits.  Requests
  * with Nq * ceil4(max_nvis) above that capacity return CSA_ERR_SCRATCH_CAPACITY before anything
- * is launched.  No cudaMalloc, cudaFree or allocating library routine is called.
+ * is launched.  No cudaMalloc, cudaFree or allocating library routine is called.  An empty
+ * batch (Nq = 0) is checked like any other and returns CSA_OK without touching the device.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  *     with that device current); make that first call before any stream capture begins.
  *   - All calls on a device share the one array, which keeps the last call's contents.  Nothing

@@ -100,6 +100,35 @@ def test_indexer_and_attention_reject_bad_arguments(C):
     assert C.hybrid_attn_decode_workspace_size(2, 4, 128, 0, 32, 50, False) > 0
 
 
+def test_empty_inputs_return_ok_before_any_launch(C):
+    """Calls with nothing to compute return CSA_OK after their argument checks and without
+    touching the device (this host has none): no complete compression block, zero rows to
+    quantise, no queries, no tokens, no sequences, no glue rows."""
+    L = C.lib()
+    f = FAKE
+    kv = C._KvRows(0x100000, 0x200000, 0x300000, 0, 512, 64)
+    f4 = C._Fp4Rows(0x100000, 0x200000, 0, 128)
+    assert L.csa_compress(f, f, f, f, f, 3, 128, 4, C.CSA_F32, f, C.CSA_F32, None, None, None) == C.CSA_OK
+    assert L.hca_compress(f, f, f, 127, 512, 128, C.CSA_BF16, f, C.CSA_F32, None, None) == C.CSA_OK
+    assert L.csa_quantize_kv(f, C.CSA_F32, 0, 512, 64, ctypes.byref(kv), None) == C.CSA_OK
+    assert L.csa_quantize_fp4(f, C.CSA_F32, 0, 128, ctypes.byref(f4), None) == C.CSA_OK
+    q4 = C._Fp4Rows(0x100000, 0x200000, 0, 128)
+    k4 = C._Fp4Rows(0x100000, 0x200000, 1000, 128)
+    for fn in (L.indexer_topk, L.indexer_topk_static):
+        tail = (None, 0, None) if fn is L.indexer_topk else (None,)
+        assert fn(ctypes.byref(q4), f, ctypes.byref(k4), C.CSA_FP4, f, f, 1000, 0, 64, 128, 4, 1024, 250,
+                  f, None, *tail) == C.CSA_OK
+        # the checks still run on an empty batch
+        assert fn(ctypes.byref(q4), f, ctypes.byref(k4), C.CSA_FP4, f, f, 1000, 0, 64, 128, 4, 0, 250,
+                  f, None, *tail) == C.CSA_ERR_UNSUPPORTED
+    assert L.hybrid_attn_prefill(f, f, f, 0, None, 0, f, 1.0, 0, 64, 512, 128, 128, C.CSA_BF16, f, None,
+                                 None) == C.CSA_OK
+    win = C._KvRows(0x100000, 0x200000, 0x300000, 0, 512, 64)
+    comp = C._KvRows(0x100000, 0x200000, 0x300000, 0, 512, 64)
+    assert L.hybrid_attn_decode(f, ctypes.byref(comp), f, f, ctypes.byref(win), f, f, 1024, f, 1.0, 0, 64, 512,
+                                4, 128, 0, f, None, None, 0, None) == C.CSA_OK
+
+
 def test_device_error_rejects_null(C):
     assert C.lib().csa_device_error(None, None) == C.CSA_ERR_INVALID_ARG
 
