@@ -209,8 +209,8 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
     a.scores = reinterpret_cast<float *>(base);
     a.idx_out = idx_out;
     a.score_out = score_out;
-    a.err = dev_error_word();
     if (Nq == 0) return CSA_OK;
+    a.err = dev_error_word();
     if (decode_indexer_eligible(a)) // FP4, 64 x 128: fused tensor-core scan + chunked top-k
         return status_of(launch_indexer_decode(a, reinterpret_cast<void *>(base), S(stream)));
     bool handled = false;
@@ -234,9 +234,9 @@ int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, i
     if (c != 32 && c != 64 && c != 128 && c != 256 && c != 512) return CSA_ERR_UNSUPPORTED;
     if (!std::isfinite(scale)) return CSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(x_win) || (kv_comp && !aligned16(kv_comp)) || !aligned16(o)) return CSA_ERR_INVALID_ARG;
+    if (T == 0) return CSA_OK;
     PrefillArgs a{q, x_win, kv_comp, n_comp, idx, idx ? k : 0, sink, scale, T, H, c, m, W, dtype, o, lse,
                   dev_error_word()};
-    if (T == 0) return CSA_OK;
     bool handled = false;
     cudaError_t e = launch_attn_prefill_tc(a, S(stream), &handled);
     if (handled) return status_of(e);
