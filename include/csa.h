@@ -106,8 +106,10 @@ typedef struct csa_fp4_rows {
  *   out      [floor(T/m), c] in `out_dtype` (CSA_F32 or CSA_BF16)
  *   out_kv   mixed FP8/BF16 rows (quantise-on-write), out_kv->n >= floor(T/m), ->c == c
  *   out_fp4  FP4 rows (quantise-on-write, for index keys), ->n >= floor(T/m), ->d == c
- * Errors: CSA_ERR_INVALID_ARG for null inputs, m out of range, c not supported, or a cache
- * whose shape does not match.
+ * Errors: CSA_ERR_INVALID_ARG for a null input, T < 0, m outside [1, 64], a dtype other than
+ * CSA_F32 / CSA_BF16, no output while floor(T/m) > 0, an input or `out` not 16-byte aligned,
+ * or an output row struct whose shape or alignment does not match; CSA_ERR_UNSUPPORTED for c
+ * not a multiple of 4 in [4, 2048].
  */
 int csa_compress(const void *Ca, const void *Cb, const void *Za, const void *Zb, const float *B,
                  int64_t T, int32_t c, int32_t m, int32_t in_dtype, void *out, int32_t out_dtype,
@@ -118,7 +120,8 @@ int csa_compress(const void *Ca, const void *Cb, const void *Za, const void *Zb,
  * the per-channel softmax pooling of tokens i*m .. i*m+m-1 with logits Z[p,d] + B[p-i*m,d].
  * No overlap; a trailing partial block is not emitted.
  *   C, Z [T, c] in `in_dtype`;  B [m, c] fp32;  1 <= m <= 1024.
- * Outputs as for csa_compress (out, out_kv; at least one non-NULL).
+ * Outputs as for csa_compress (out, out_kv; at least one non-NULL).  Errors as for
+ * csa_compress, with m outside [1, 1024].
  */
 int hca_compress(const void *C, const void *Z, const float *B, int64_t T, int32_t c, int32_t m,
                  int32_t in_dtype, void *out, int32_t out_dtype, const csa_kv_rows *out_kv,
@@ -129,6 +132,9 @@ int hca_compress(const void *C, const void *Z, const float *B, int64_t T, int32_
  * csa_kv_rows ([ledger]).  Per row: s = amax(|x[0:c-rope]|) / 448 (fp32 division; s = 1 when
  * that is not positive), fp8 = e4m3(x / s) rounded to nearest even and saturated at 448,
  * rope = bf16(x[c-rope:c]) rounded to nearest even.
+ * Errors: CSA_ERR_INVALID_ARG for a null x or out, n < 0, a dtype other than CSA_F32 /
+ * CSA_BF16, c outside [1, 4096], x not 16-byte aligned, out->rope_dims != rope_dims, or an
+ * `out` that does not hold n rows of c channels as described above.
  */
 int csa_quantize_kv(const void *x, int32_t in_dtype, int64_t n, int32_t c, int32_t rope_dims,
                     const csa_kv_rows *out, void *stream);
@@ -137,6 +143,8 @@ int csa_quantize_kv(const void *x, int32_t in_dtype, int64_t n, int32_t c, int32
  * csa_quantize_fp4 -- write rows x [n, d] (`in_dtype`) as FP4 rows.  Per block of 32: the scale
  * exponent is the smallest e with amax <= 6 * 2^e (clamped to [-127, 127]; -127 for an all-zero
  * block), element = e2m1(x / 2^e) rounded to nearest even, every zero encoded as +0.
+ * Errors: CSA_ERR_INVALID_ARG for a null x, n < 0, a dtype other than CSA_F32 / CSA_BF16, d not
+ * a positive multiple of 32, x not 16-byte aligned, or an `out` that does not hold n rows of d.
  */
 int csa_quantize_fp4(const void *x, int32_t in_dtype, int64_t n, int32_t d,
                      const csa_fp4_rows *out, void *stream);
@@ -163,6 +171,11 @@ int csa_quantize_fp4(const void *x, int32_t in_dtype, int64_t n, int32_t d,
  *            -inf in padded slots)
  *   ws       workspace of at least indexer_topk_workspace_size(Nq, max_nvis, k) bytes
  * Limits: 1 <= k <= 2048, 1 <= H_I <= 128, d_I a multiple of 32 (FP4) or 8 and <= 512.
+ * Errors: CSA_ERR_INVALID_ARG for a null q, w, keys or idx_out, Nq < 0, n_keys < 0, m < 1,
+ * max_nvis < 0, an unknown fmt, w (or dense q / keys) not 16-byte aligned, or FP4 rows that do
+ * not hold Nq*H_I query rows / n_keys key rows of d_I (d_I a multiple of 32);
+ * CSA_ERR_UNSUPPORTED for k, H_I or d_I outside the limits or max_nvis > 8,388,480;
+ * CSA_ERR_WORKSPACE when Nq > 0 and ws is NULL or smaller than the size above.
  */
 size_t indexer_topk_workspace_size(int64_t Nq, int64_t max_nvis, int32_t k);
 int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
@@ -211,7 +224,11 @@ int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t
  *   idx [T, k] int32 or NULL; negative entries (padding) are skipped, entries >= n_comp are
  *            skipped and set CSA_DEVERR_INDEX
  *   sink [H] fp32 (-inf allowed: no sink);  o [T, H, c] in `dtype`;  lse [T, H] fp32 or NULL
- * Limits: c a multiple of 32 and <= 512, 1 <= H <= 128, 1 <= W <= 1024, k <= 4096.
+ * Limits: c one of 32, 64, 128, 256, 512; 1 <= H <= 128; 1 <= W <= 1024; 0 <= k <= 4096.
+ * Errors: CSA_ERR_INVALID_ARG for a null q, x_win, sink or o, T < 0, n_comp < 0, m < 1, a
+ * dtype other than CSA_F32 / CSA_BF16, a NULL kv_comp with n_comp > 0, idx with k outside
+ * [0, 4096], a non-finite scale, or q, x_win, kv_comp or o not 16-byte aligned;
+ * CSA_ERR_UNSUPPORTED for c, H or W outside the limits.
  */
 int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, int64_t n_comp,
                         const int32_t *idx, int32_t k, const float *sink, float scale, int64_t T,
@@ -230,7 +247,13 @@ int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, i
  *            s < min(N_vis, max_nvis))
  *   o        [B, H, c] bf16;  lse [B, H] fp32 or NULL
  *   ws       workspace of hybrid_attn_decode_workspace_size(...) bytes (split-K partials)
- * Limits: c a multiple of 32 and <= 512, H <= 128, W <= 1024.
+ * Limits: c one of 32, 64, 128, 256, 512; 1 <= H <= 128; 1 <= W <= 1024; 1 <= k <= 4096 with
+ * idx; W + (k or max_nvis) <= 2^30.
+ * Errors: CSA_ERR_INVALID_ARG for a null q, comp, comp_off, pos, win, win_len, sink or o,
+ * B < 0, m < 1, max_nvis < 0, idx with k outside the limits, a non-finite scale, row structs
+ * that do not match c (or, for win, hold fewer than B*W rows), or q / o not 16-byte aligned;
+ * CSA_ERR_UNSUPPORTED for c, H, W or the key count outside the limits; CSA_ERR_WORKSPACE when
+ * ws is NULL or smaller than the size above.
  */
 size_t hybrid_attn_decode_workspace_size(int32_t B, int32_t H, int32_t c, int32_t k, int32_t W,
                                          int64_t max_nvis, int32_t use_idx);
