@@ -1,6 +1,7 @@
 // abi.cu -- the extern "C" entry points of libcsa: host-side argument checks, workspace
 // carving and dispatch to the kernels.  No allocation, no synchronisation (except
 // csa_device_error), no CPU fallback: every step of the path runs in this library's kernels.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -9,17 +10,21 @@
 namespace csa {
 __device__ int g_dev_error = 0;
 
+// Device address of g_dev_error for the current device, looked up once per device; callers on
+// several host threads may race on the first lookup, and all of them store the same address.
 int *dev_error_word()
 {
-    static int *addr[64] = {nullptr};
+    static std::atomic<int *> addr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
+    int *a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int *>(p);
+        a = static_cast<int *>(p);
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 cudaError_t launch_attn_prefill_generic(const PrefillArgs &a, cudaStream_t st);
 cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled);
