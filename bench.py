@@ -88,32 +88,109 @@ def attn_flops(T, H, c, W, m, n_comp, k=None) -> float:
 # ---------------------------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock, its maximum and the active clock-event reasons of the bench's GPU, sampled while
+    the timed region runs.  NVML is polled every 2 ms from a background thread (one sample is
+    also taken on entry and one on exit), so a timed region of a few milliseconds still holds
+    samples; without NVML, nvidia-smi samples at its 200 ms minimum period.  The GPU is found by
+    its PCI address when the caller passes one (CUDA and NVML may number devices differently),
+    else by index.  Only reads the GPU's state."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pci=None, period_s: float = 0.002, nvml=None):
         self.gpu = gpu_index
+        self.pci = pci                  # (domain, bus, device) or None
+        self.period = period_s
+        self._nvml_mod = nvml           # a stand-in module for tests; pynvml otherwise
         self.proc = None
-        self.lines = []
+        self.lines = []                 # nvidia-smi csv lines
+        self.samples = []               # NVML samples: (sm_mhz, max_mhz, reasons)
+        self.source = None
+        self._nv = self._h = None
+        self._stop = threading.Event()
+        self._t = None
+
+    # -- NVML ---------------------------------------------------------------------------------
+    def _nvml_open(self):
+        try:
+            nv = self._nvml_mod
+            if nv is None:
+                import pynvml as nv
+            nv.nvmlInit()
+        except Exception:
+            return False
+        h = None
+        if self.pci is not None:
+            try:
+                h = nv.nvmlDeviceGetHandleByPciBusId("%08x:%02x:%02x.0" % tuple(self.pci))
+            except Exception:
+                h = None
+        try:
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self._max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+            return False
+        self._nv, self._h = nv, h
+        return True
+
+    def _nvml_sample(self):
+        nv, h = self._nv, self._h
+        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+        self.samples.append((sm, self._max, [n for n, b in self.REASONS if bits & b]))
+
+    def _nvml_loop(self):
+        while not self._stop.wait(self.period):
+            try:
+                self._nvml_sample()
+            except Exception:
+                return
+
+    # -- nvidia-smi ---------------------------------------------------------------------------
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
 
     def __enter__(self):
+        if self._nvml_open():
+            self.source = "nvml"
+            self._nvml_sample()
+            self._t = threading.Thread(target=self._nvml_loop, daemon=True)
+            self._t.start()
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
+            self.source = "nvidia-smi"
         except Exception:
             self.proc = None
         time.sleep(0.3)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join(timeout=5)
+            try:
+                self._nvml_sample()
+            except Exception:
+                pass
+            try:
+                self._nv.nvmlShutdown()
+            except Exception:
+                pass
+            self._nv = None
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -124,7 +201,11 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s_mhz, m_mhz, rs in self.samples:
+            sm.append(s_mhz)
+            mx.append(m_mhz)
+            reasons.update(rs)
+        names = [n for n, _ in self.REASONS]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
@@ -138,9 +219,10 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "source": self.source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -471,20 +553,31 @@ WORKLOADS = {"hca_prefill_32k": HcaPrefill, "csa_prefill_64k": CsaPrefill, "csa_
 
 class OracleHca:
     """The oracle on a bounded sample of the HCA layer: the full compression (amortised over T)
-    plus attention of n_tokens query tokens evenly spaced over the sequence.  Inputs are drawn
-    once (untimed); run() times the oracle's own work."""
+    plus attention of about n_tokens query tokens, taken as whole groups of G consecutive tokens
+    (G = the rows of one seeded block of q, so no drawn row is wasted) spread evenly over the
+    sequence, so the sample spans every key count of the layer.  Inputs are drawn untimed;
+    run() times the oracle's own work, calling the attention on chunks of at most 1024 tokens
+    so the host memory it holds stays bounded."""
+    CHUNK = 1024
 
     def __init__(self, w, n_tokens: int, seed_rank: int = 0):
         T, c, H, m = w.T, w.c, w.H, w.m
-        self.w, self.n = w, n_tokens
+        self.w, self.seed_rank = w, seed_rank
+        self.G = WL.block_rows_for(H * c)
+        n_blocks = max(1, T // self.G)
+        n_groups = max(1, min(n_blocks, -(-int(n_tokens) // self.G)))
+        self.starts = np.unique(np.linspace(0, n_blocks - 1, n_groups).round().astype(np.int64)) * self.G
+        self.n = int(sum(min(self.G, T - s) for s in self.starts))
         self.Cc = WL.draw(w, "C", 0, T, seq=seed_rank)
         self.Z = WL.draw(w, "Z", 0, T, seq=seed_rank)
         self.B = WL.normal_rows(w.seed, f"B/L0/S{seed_rank}", c, 0, m, std=w.bias_std)
-        self.rows = np.linspace(0, T - 1, n_tokens).astype(np.int64)
-        self.qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1, seq=seed_rank)[0]
-                            for t in self.rows]).reshape(n_tokens, H, c)
         self.X = WL.draw(w, "X", 0, T, seq=seed_rank)
         self.sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
+
+    def _chunks(self):
+        per = max(1, self.CHUNK // self.G)
+        for i in range(0, len(self.starts), per):
+            yield self.starts[i:i + per]
 
     def run(self):
         """Returns (tokens/s, seconds of oracle work, compress seconds, attention seconds)."""
@@ -492,15 +585,23 @@ class OracleHca:
         w = self.w
         t0 = time.perf_counter()
         KV = O.hca_compress(self.Cc, self.Z, self.B, w.m)
-        t1 = time.perf_counter()
-        O.hybrid_attn_prefill(self.qs, self.X, KV, self.sink, 1.0, w.m, w.W, rows=self.rows)
-        t2 = time.perf_counter()
-        per_token = (t1 - t0) / w.T + (t2 - t1) / self.n
-        return 1.0 / per_token, t2 - t0, t1 - t0, t2 - t1
+        t_comp = time.perf_counter() - t0
+        t_attn = 0.0
+        for starts in self._chunks():
+            ends = [min(int(s) + self.G, w.T) for s in starts]
+            rows = np.concatenate([np.arange(int(s), e) for s, e in zip(starts, ends)])
+            qs = np.concatenate([WL.draw(w, "q", int(s), e, seq=self.seed_rank) for s, e in zip(starts, ends)])
+            qs = qs.reshape(len(rows), w.H, w.c)
+            t1 = time.perf_counter()
+            O.hybrid_attn_prefill(qs, self.X, KV, self.sink, 1.0, w.m, w.W, rows=rows)
+            t_attn += time.perf_counter() - t1
+        per_token = t_comp / w.T + t_attn / self.n
+        return 1.0 / per_token, t_comp + t_attn, t_comp, t_attn
 
     def describe(self):
         return (f"full hca_compress of T={self.w.T} (amortised per token) + hybrid attention of {self.n} "
-                f"query tokens evenly spaced over the layer")
+                f"query tokens ({len(self.starts)} groups of {self.G} consecutive tokens evenly spaced over "
+                f"the layer)")
 
 
 class OracleDecode:
@@ -605,13 +706,33 @@ class OracleMixed:
 
 
 def oracle_hca_sample(w, target_s: float = 10.0):
-    """cpu_baseline leg: calibrate the sample so the oracle's attention work takes ~target_s."""
-    probe = OracleHca(w, 16)
-    _, _, _, t_attn = probe.run()
-    n = int(min(4096, max(16, target_s / max(t_attn / 16, 1e-6))))
+    """cpu_baseline leg: size the sample so the oracle's work takes about target_s.  Two probes
+    (one group of tokens, then four) give the attention's cost per token apart from its fixed
+    cost per call; the sample is then as many tokens as fill the target, at most the layer."""
+    g = WL.block_rows_for(w.H * w.c)
+    t1 = OracleHca(w, g).run()[3]
+    probe = OracleHca(w, 4 * g)
+    t4 = probe.run()[3]
+    per_token = max((t4 - t1) / (3 * g), t4 / (4 * g) / 4, 1e-7)
+    per_chunk = max(t1 - g * per_token, 0.0)
+    chunk_tokens = OracleHca.CHUNK
+    n = int(max(g, min(w.T, target_s / (per_token + per_chunk / chunk_tokens))))
     job = OracleHca(w, n)
     tps, secs, _, _ = job.run()
     return tps, secs, job.describe()
+
+
+def oracle_repeat(job, target_s: float = 10.0, max_reps: int = 20):
+    """cpu_baseline leg for a sample that is small next to target_s: time job.run() again until
+    the oracle has worked about target_s.  Returns (tokens/s over all runs, seconds, runs)."""
+    tokens = secs = 0.0
+    reps = 0
+    while reps < max_reps and (reps == 0 or secs < target_s):
+        tps_i, s_i = job.run()[:2]
+        tokens += tps_i * s_i
+        secs += s_i
+        reps += 1
+    return tokens / secs, secs, reps
 
 
 # ---------------------------------------------------------------------------------------------
@@ -662,7 +783,9 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    props = torch.cuda.get_device_properties(local)
+    pci = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    with ClockSampler(local, pci) as clk:
         start.record(stream)
         for i in range(args.steps):
             job.step(evs[i])
@@ -751,8 +874,8 @@ def main():
                 tps, secs, desc = oracle_hca_sample(w)
             else:
                 job_o = OracleDecode(w, 4) if args.workload == "csa_decode_1m" else OracleMixed(w, 8)
-                tps, secs = job_o.run()
-                desc = job_o.describe()
+                tps, secs, reps = oracle_repeat(job_o)
+                desc = f"{job_o.describe()}; the sample timed {reps} times over"
             line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
                                     "sample": desc, "seconds": secs}
         print(json.dumps(line), flush=True)
