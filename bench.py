@@ -22,6 +22,7 @@ cpu_baseline = the fp64 oracle timed on this host's cores on a bounded sample.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import json
 import os
 import statistics
@@ -226,6 +227,46 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
+# CUDA-event spans of the library calls inside a step
+# ---------------------------------------------------------------------------------------------
+
+class Spans:
+    """Start/end CUDA events around each named library call of one step, recorded on the current
+    stream.  The events are created ahead of time (prepare), so a step can be captured into a
+    CUDA graph with its spans; ms(name) sums the spans of that name."""
+
+    def __init__(self, torch):
+        self.torch = torch
+        self.pairs = {}
+        self.pool = []
+        self.i = 0
+
+    def prepare(self, job, pairs: int = 32):
+        self.pool = [self.torch.cuda.Event(enable_timing=True) for _ in range(2 * pairs)]
+
+    def take(self):
+        if self.i < len(self.pool):
+            self.i += 1
+            return self.pool[self.i - 1]
+        return self.torch.cuda.Event(enable_timing=True)
+
+    def ms(self, name: str) -> float:
+        return sum(s.elapsed_time(e) for s, e in self.pairs.get(name, []))
+
+
+@contextlib.contextmanager
+def span(sp, name: str):
+    if sp is None:
+        yield
+        return
+    s, e = sp.take(), sp.take()
+    s.record()
+    yield
+    e.record()
+    sp.pairs.setdefault(name, []).append((s, e))
+
+
+# ---------------------------------------------------------------------------------------------
 # workloads on the GPU
 # ---------------------------------------------------------------------------------------------
 
@@ -263,15 +304,16 @@ class HcaPrefill:
         self.flops = attn_flops(T, H, c, w.W, m, T // m)
         self.tokens = T
         self.launches_per_step = 2
+        # (name, bound, algorithmic work per step): the first is the dominant kernel
+        self.kernels = [("hybrid_attn_prefill", "tensor", self.flops)]
+        self.step_work = ("tensor", self.flops)
 
-    def step(self, ev=None):
+    def step(self, sp=None):
         C = self.C
-        C.hca_compress(self.Cc, self.Z, self.B, self.w.m, out=self.kv)
-        if ev is not None:
-            ev[0].record()
-        C.hybrid_attn_prefill(self.q, self.X, self.kv, self.sink, self.scale, self.w.m, self.w.W, o=self.o)
-        if ev is not None:
-            ev[1].record()
+        with span(sp, "hca_compress"):
+            C.hca_compress(self.Cc, self.Z, self.B, self.w.m, out=self.kv)
+        with span(sp, "hybrid_attn_prefill"):
+            C.hybrid_attn_prefill(self.q, self.X, self.kv, self.sink, self.scale, self.w.m, self.w.W, o=self.o)
 
     # end-to-end through the C ABI: pinned host inputs -> device -> compute -> host output
     def setup_e2e(self):
@@ -327,19 +369,19 @@ class CsaPrefill:
         self.flops_attn = attn_flops(T, H, c, w.W, m, n, w.k)
         self.tokens = T
         self.launches_per_step = 5  # compress x2, indexer scores, top-k, attention
-        self.kernel_name = "indexer_topk (scores)"
+        self.kernels = [("indexer_topk", "tensor", self.flops), ("hybrid_attn_prefill", "tensor", self.flops_attn)]
+        self.step_work = ("tensor", self.flops + self.flops_attn)
 
-    def step(self, ev=None):
+    def step(self, sp=None):
         C, w = self.C, self.w
-        C.csa_compress(*self.kv_in, self.B, w.m, out=self.kvc)
-        C.csa_compress(*self.ki_in, self.BI, w.m, out=self.keys)
-        if ev is not None:
-            ev[0].record()
-        C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=w.T // w.m, idx_out=self.idx,
-                       workspace=self.ws)
-        if ev is not None:
-            ev[1].record()
-        C.hybrid_attn_prefill(self.q, self.X, self.kvc, self.sink, 1.0, w.m, w.W, idx=self.idx, o=self.o)
+        with span(sp, "csa_compress"):
+            C.csa_compress(*self.kv_in, self.B, w.m, out=self.kvc)
+            C.csa_compress(*self.ki_in, self.BI, w.m, out=self.keys)
+        with span(sp, "indexer_topk"):
+            C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=w.T // w.m, idx_out=self.idx,
+                           workspace=self.ws)
+        with span(sp, "hybrid_attn_prefill"):
+            C.hybrid_attn_prefill(self.q, self.X, self.kvc, self.sink, 1.0, w.m, w.W, idx=self.idx, o=self.o)
 
     def setup_e2e(self):
         torch = self.torch
@@ -401,21 +443,22 @@ class CsaDecode1M:
         self.o = torch.empty_like(self.q)
         torch.cuda.synchronize()
         self.bytes = float(Bn * nv * (di // 2 + di // 32))           # FP4 key scan (dominant)
-        self.bytes_step = self.bytes + Bn * (w.k + W) * (c - w.rope + 2 * w.rope + 4) + 2 * Bn * H * c * 2
+        row = c - w.rope + 2 * w.rope + 4                              # 580 B per FP8/BF16 cache row
+        self.bytes_attn = float(Bn * (min(w.k, nv) + W) * row + 2 * Bn * H * c * 2)  # gathered rows + q, o
+        self.bytes_step = self.bytes + self.bytes_attn
         self.tokens = Bn
         self.launches_per_step = 4
-        self.kernel_name = "indexer_topk (FP4 scan + top-k)"
+        self.kernels = [("indexer_topk", "hbm", self.bytes), ("hybrid_attn_decode", "hbm", self.bytes_attn)]
+        self.step_work = ("hbm", self.bytes_step)
 
-    def step(self, ev=None):
+    def step(self, sp=None):
         C, w = self.C, self.w
-        if ev is not None:
-            ev[0].record()
-        C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=self.nv, q_pos=self.pos,
-                       key_off=self.key_off, idx_out=self.idx, workspace=self.ws)
-        if ev is not None:
-            ev[1].record()
-        C.hybrid_attn_decode(self.q, self.comp, self.key_off, self.pos, self.win, self.win_len, self.sink, 1.0,
-                             w.m, w.W, max_nvis=self.nv, idx=self.idx, o=self.o, workspace=self.wsd)
+        with span(sp, "indexer_topk"):
+            C.indexer_topk(self.qI, self.wI, self.keys, w.m, w.k, max_nvis=self.nv, q_pos=self.pos,
+                           key_off=self.key_off, idx_out=self.idx, workspace=self.ws)
+        with span(sp, "hybrid_attn_decode"):
+            C.hybrid_attn_decode(self.q, self.comp, self.key_off, self.pos, self.win, self.win_len, self.sink, 1.0,
+                                 w.m, w.W, max_nvis=self.nv, idx=self.idx, o=self.o, workspace=self.wsd)
 
     def setup_e2e(self):
         torch = self.torch
@@ -501,30 +544,37 @@ class MixedDecode:
             qx = np.concatenate([WL.draw(w, "qI", 0, 1, layer=0, seq=seqs[b]).reshape(Hi, di) for b in range(Bn)])
             C.csa_quantize_fp4(torch.from_numpy(qx).to(device), self.layers[0].qI)
         torch.cuda.synchronize()
-        first = next(L for L in self.layers if L.csa)
-        self.bytes = float(first.nv.sum() * (di // 2 + di // 32))   # FP4 key scan of one CSA layer
-        self.tokens = Bn
+        # algorithmic bytes per step: FP4 key scans of the CSA layers, the gathered (CSA: window +
+        # top-k) or streamed (HCA: window + every visible entry) 580-byte cache rows, q and o
+        row = c - w.rope + 2 * w.rope + 4
+        qo = 2 * Bn * H * c * 2
+        self.bytes_scan = float(sum(L.nv.sum() * (di // 2 + di // 32) for L in self.layers if L.csa))
+        self.bytes_attn = float(sum((np.minimum(L.nv, w.k).sum() if L.csa else L.nv.sum()) * row + Bn * W * row + qo
+                                    for L in self.layers))
+        self.bytes_glue = float((len(self.layers) - 1) * (2 * Bn * H * c * 2 + c * c * 2)
+                                + sum(Bn * Hi * (di // 2 + di // 32) + di * c * 2 for L in self.layers[1:] if L.csa))
+        self.bytes_step = self.bytes_scan + self.bytes_attn + self.bytes_glue
+        self.tokens = Bn * len(self.layers)   # sequence-layers completed per step
         self.launches_per_step = sum(4 if L.csa else 2 for L in self.layers) + len(self.layers) - 1
-        self.kernel_name = "indexer_topk (FP4 scan + top-k), first CSA layer"
+        self.kernels = [("indexer_topk", "hbm", self.bytes_scan), ("hybrid_attn_decode", "hbm", self.bytes_attn),
+                        ("csa_decode_glue", "hbm", self.bytes_glue)]
+        self.step_work = ("hbm", self.bytes_step)
 
-    def step(self, ev=None):
+    def step(self, sp=None):
         C, w = self.C, self.w
         q = self.q0
-        timed = False
         for l, L in enumerate(self.layers):
             if L.csa:
-                if ev is not None and not timed:
-                    ev[0].record()
-                C.indexer_topk(L.qI, L.wI, L.keys, L.m, w.k, max_nvis=L.max_nv, q_pos=self.pos, key_off=L.off,
-                               idx_out=L.idx, workspace=L.ws)
-                if ev is not None and not timed:
-                    ev[1].record()
-                    timed = True
-            C.hybrid_attn_decode(q, L.comp, L.off, self.pos, L.win, self.win_len, L.sink, 1.0, L.m, w.W,
-                                 max_nvis=L.max_nv, idx=L.idx if L.csa else None, o=L.o, workspace=L.wsd)
+                with span(sp, "indexer_topk"):
+                    C.indexer_topk(L.qI, L.wI, L.keys, L.m, w.k, max_nvis=L.max_nv, q_pos=self.pos, key_off=L.off,
+                                   idx_out=L.idx, workspace=L.ws)
+            with span(sp, "hybrid_attn_decode"):
+                C.hybrid_attn_decode(q, L.comp, L.off, self.pos, L.win, self.win_len, L.sink, 1.0, L.m, w.W,
+                                     max_nvis=L.max_nv, idx=L.idx if L.csa else None, o=L.o, workspace=L.wsd)
             if l + 1 < len(self.layers):
                 nxt = self.layers[l + 1]
-                C.csa_decode_glue(L.o, L.P, L.Rm, q_next=L.q_next, qI=nxt.qI if nxt.csa else None)
+                with span(sp, "csa_decode_glue"):
+                    C.csa_decode_glue(L.o, L.P, L.Rm, q_next=L.q_next, qI=nxt.qI if nxt.csa else None)
                 q = L.q_next
 
     def setup_e2e(self):
@@ -722,6 +772,66 @@ def oracle_hca_sample(w, target_s: float = 10.0):
     return tps, secs, job.describe()
 
 
+class OracleCsa:
+    """The oracle on a bounded sample of the CSA layer prefill: the full compression of the KV
+    entries and of the index keys (amortised over T), then, for groups of G consecutive query
+    tokens spread evenly over the layer, the indexer over every visible entry, the top-k and the
+    hybrid attention over window + selected entries.  Inputs are drawn untimed."""
+
+    def __init__(self, w, n_groups: int, seed_rank: int = 0):
+        T, c, m, di = w.T, w.c, w.m, w.d_I
+        self.w, self.seed_rank = w, seed_rank
+        self.G = WL.block_rows_for(w.H * w.c)
+        n_blocks = max(1, T // self.G)
+        self.starts = np.unique(np.linspace(0, n_blocks - 1, max(1, min(n_blocks, n_groups))).round()
+                                .astype(np.int64)) * self.G
+        self.n = int(sum(min(self.G, T - s) for s in self.starts))
+        self.kv_in = [WL.draw(w, nm, 0, T, seq=seed_rank) for nm in ("Ca", "Cb", "Za", "Zb")]
+        self.ki_in = [WL.draw(w, nm, 0, T, seq=seed_rank) for nm in ("CIa", "CIb", "ZIa", "ZIb")]
+        self.B = WL.normal_rows(w.seed, f"B/L0/S{seed_rank}", c, 0, 2 * m, std=w.bias_std)
+        self.BI = WL.normal_rows(w.seed, f"BI/L0/S{seed_rank}", di, 0, 2 * m, std=w.bias_std)
+        self.X = WL.draw(w, "X", 0, T, seq=seed_rank)
+        self.sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
+        self.rows = [np.arange(int(s), min(int(s) + self.G, T)) for s in self.starts]
+        self.q = [WL.draw(w, "q", int(r[0]), int(r[-1]) + 1, seq=seed_rank).reshape(len(r), w.H, c) for r in self.rows]
+        self.qI = [WL.qI_lowrank(w, int(r[0]), int(r[-1]) + 1).reshape(len(r), w.H_I, di) for r in self.rows]
+        self.wI = [WL.draw(w, "w", int(r[0]), int(r[-1]) + 1, seq=seed_rank) for r in self.rows]
+
+    def run(self):
+        """Returns (tokens/s, seconds of oracle work, compress seconds, per-token seconds)."""
+        import oracle as O
+        w = self.w
+        t0 = time.perf_counter()
+        KV = O.csa_compress(*self.kv_in, self.B, w.m)
+        KI = O.csa_compress(*self.ki_in, self.BI, w.m)
+        t_comp = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        for rows, q, qI, wI in zip(self.rows, self.q, self.qI, self.wI):
+            idx, _ = O.indexer_topk(qI, wI, KI, rows, w.m, w.k)
+            by_pos = {int(t): idx[i] for i, t in enumerate(rows)}   # the oracle looks rows up by position
+            O.hybrid_attn_prefill(q, self.X, KV, self.sink, 1.0, w.m, w.W, idx=by_pos, rows=rows)
+        t_tok = time.perf_counter() - t1
+        per_token = t_comp / w.T + t_tok / self.n
+        return 1.0 / per_token, t_comp + t_tok, t_comp, t_tok
+
+    def describe(self):
+        return (f"full csa_compress of the KV entries and the index keys (T={self.w.T}, amortised per token) + "
+                f"indexer over every visible entry, top-{self.w.k} and hybrid attention of {self.n} query tokens "
+                f"({len(self.starts)} groups of {self.G} consecutive tokens evenly spaced over the layer)")
+
+
+def oracle_csa_sample(w, target_s: float = 10.0):
+    """cpu_baseline leg of the CSA prefill: one probe group gives the cost per group; the sample
+    then takes as many evenly spaced groups as fill about target_s."""
+    probe = OracleCsa(w, 2)
+    _, _, t_comp, t_tok = probe.run()
+    per_group = t_tok / len(probe.starts)
+    n = int(max(2, min(w.T // probe.G, (target_s - t_comp) / max(per_group, 1e-6))))
+    job = OracleCsa(w, n)
+    tps, secs, _, _ = job.run()
+    return tps, secs, job.describe()
+
+
 def oracle_repeat(job, target_s: float = 10.0, max_reps: int = 20):
     """cpu_baseline leg for a sample that is small next to target_s: time job.run() again until
     the oracle has worked about target_s.  Returns (tokens/s over all runs, seconds, runs)."""
@@ -737,28 +847,252 @@ def oracle_repeat(job, target_s: float = 10.0, max_reps: int = 20):
 
 # ---------------------------------------------------------------------------------------------
 
+DEFAULT_WORKLOADS = ("hca_prefill_32k", "csa_prefill_64k", "csa_decode_1m", "mixed_decode_64")
+
+
+def check_world(gpus: int, world: int):
+    """--gpus N must match the number of ranks the launcher started (one process per GPU):
+    returns None when it does, else the reason to refuse the run."""
+    if gpus < 1:
+        return f"--gpus must be at least 1 (got {gpus})"
+    if gpus != world:
+        return (f"--gpus {gpus} but WORLD_SIZE={world}: launch one process per GPU, e.g. "
+                f"python -m torch.distributed.run --nproc-per-node {gpus} --master-addr 127.0.0.1 bench.py --gpus {gpus}")
+    return None
+
+
+def traffic_table(path=None):
+    """DRAM bytes per launch of the dominant kernels, from ncu captures summarised in
+    profiles/dram_traffic.md: {(workload, kernel): (bytes, source sha256 prefix, source file)}."""
+    path = path or os.path.join(ROOT, "profiles", "dram_traffic.md")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    for ln in open(path):
+        parts = [p.strip() for p in ln.strip().strip("|").split("|")]
+        if len(parts) < 5 or not parts[3].replace(".", "").replace("e", "").replace("+", "").isdigit():
+            continue
+        wl, kern, src, nbytes, sha = parts[:5]
+        out[(wl, kern)] = (float(nbytes), sha, src)
+    return out
+
+
+def source_sha(rel: str) -> str:
+    """sha256 prefix of the kernel sources a capture was taken from ('+'-joined file names under
+    csrc/, hashed in that order); empty when a file is missing."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in rel.split("+"):
+        p = os.path.join(ROOT, "compressed_sparse_kv_csa_b200", "csrc", f.strip())
+        if not os.path.exists(p):
+            return ""
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str, kernel: str):
+    """The captured DRAM bytes per launch for (workload, kernel), or None when there is no capture
+    or the kernel's source has changed since it was taken."""
+    row = traffic_table().get((workload, kernel))
+    if row is None:
+        return None
+    nbytes, sha, src = row
+    return nbytes if source_sha(src) == sha else None
+
+
+def roofline(bound, work, ms, pk, src, kernel, traffic=None):
+    if bound == "hbm":
+        ach = work / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "kernel": kernel, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "peak_source": f"{src} HBM copy", "traffic": traffic,
+                "bytes_per_launch": work, "launch_ms": ms}
+    ach = work / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": kernel, "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": ach / pk["bf16_tflops"], "peak_source": f"{src} dense bf16 burst", "traffic": traffic,
+            "flops_per_launch": work, "launch_ms": ms}
+
+
+def workload_config(name, w, job, world):
+    cfg = {"workload": name, "T": w.T, "c": w.c, "rope_dims": w.rope, "m": w.m, "H": w.H, "W": w.W,
+           "parallelism": f"replicas x{world}"}
+    if w.kind == "csa_decode":
+        cfg.update({"B": w.B, "n_comp_per_seq": (w.T + 1) // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+                    "l2": "FP4 key scan (143 MB) and KV cache (1.2 GB) larger than L2"})
+    elif w.kind == "mixed_decode":
+        cfg = {"workload": name, "B": w.B, "layers": list(w.extra["layers"]), "c": w.c,
+               "rope_dims": w.rope, "H": w.H, "W": w.W, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+               "m_csa": w.extra["m_csa"], "m_hca": w.extra["m_hca"],
+               "context": f"log-uniform [{w.extra['len_lo']}, {w.extra['len_hi']}]",
+               "total_context_tokens": int(job.lens.sum()), "parallelism": f"replicas x{world}",
+               "tokens": "sequences x layers completed per step",
+               "l2": "KV caches of the stack ({:.2f} GB) larger than L2".format(
+                   sum(L.comp.fp8.numel() + L.comp.rope.numel() * 2 + L.comp.scale.numel() * 4
+                       + (L.keys.codes.numel() + L.keys.scales.numel() if L.csa else 0)
+                       for L in job.layers) / 1e9)}
+    elif w.kind == "csa_prefill":
+        cfg.update({"n_comp": w.T // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
+                    "l2": "inputs larger than L2 (q alone is 4.3 GB)"})
+    else:
+        cfg.update({"n_comp": w.T // w.m, "l2": f"inputs larger than L2 (q alone is {w.T * w.H * w.c * 2 / 1e9:.1f} GB)"})
+    return cfg
+
+
+def capture_steps(job, steps, torch, stream):
+    """The timed region as one CUDA graph of `steps` steps, each with its own span events (the
+    library's calls only enqueue kernels, so they capture).  Returns (graph, spans per step), or
+    (None, reason) when capture is not possible."""
+    spans = [Spans(torch) for _ in range(steps)]
+    for sp in spans:   # create every event before capture
+        sp.prepare(job)
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g, stream=stream):
+            for sp in spans:
+                job.step(sp)
+    except Exception as e:  # pragma: no cover - depends on the driver
+        return None, f"{type(e).__name__}: {e}"
+    return g, spans
+
+
+def measure(name, args, world, rank, dist, device, torch, C):
+    """Time one workload: W warm-up steps, then exactly K steps in one timed region bracketed by
+    a barrier and a synchronize, SM clocks sampled during it; then the end-to-end leg."""
+    w = WL.WORKLOADS[name]
+    if args.T is not None:
+        import dataclasses
+        w = dataclasses.replace(w, T=args.T)
+    job = WORKLOADS[name](w, rank, torch, C, device)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        stream = torch.cuda.current_stream()
+        for _ in range(max(args.warmup, 3)):
+            job.step()
+        torch.cuda.synchronize()
+        graph, spans = (None, "eager (--eager)")
+        if not args.eager:
+            graph, spans = capture_steps(job, args.steps, torch, stream)
+        timing = f"one CUDA graph of the {args.steps} steps" if graph is not None else f"eager launches ({spans})"
+        if graph is None:
+            spans = [Spans(torch) for _ in range(args.steps)]
+        graph is not None and graph.replay()       # one untimed replay (graph upload)
+        torch.cuda.synchronize()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        props = torch.cuda.get_device_properties(device)
+        pci = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        with ClockSampler(device.index or 0, pci) as clk:
+            start.record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                for sp in spans:
+                    job.step(sp)
+            stop.record(stream)
+            torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = start.elapsed_time(stop) / args.steps
+        names = [k[0] for k in job.kernels]
+        try:
+            kern_ms = [sum(sp.ms(n) for sp in spans) / args.steps for n in names]
+        except RuntimeError as e:  # event timing inside the graph unavailable: spans on eager launches
+            spans = [Spans(torch) for _ in range(args.steps)]
+            for sp in spans:
+                job.step(sp)
+            torch.cuda.synchronize()
+            kern_ms = [sum(sp.ms(n) for sp in spans) / args.steps for n in names]
+            timing += f"; kernel spans from eager launches ({type(e).__name__})"
+        vals = max_over_ranks([ms] + kern_ms, world, dist, device)
+        ms, kern_ms = vals[0], vals[1:]
+        del graph
+        torch.cuda.synchronize()
+
+        # end to end through the C ABI with host buffers
+        job.setup_e2e()
+        job.step_e2e()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            job.step_e2e()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    (e2e_ms,) = max_over_ranks([e2e_ms], world, dist, device)
+    if world > 1:
+        dist.barrier()
+    pk, src = peaks()
+    kernels = {}
+    for (kname, bound, work), kms in zip(job.kernels, kern_ms):
+        kernels[kname] = roofline(bound, work, kms, pk, src, kname, traffic_for(name, kname))
+    bound, work = job.step_work
+    res = {
+        "value": world * job.tokens / (ms * 1e-3),
+        "unit": "tokens/s" if w.kind != "mixed_decode" else "tokens/s (sequence x layer)",
+        "ms_per_step": ms,
+        "config": workload_config(name, w, job, world),
+        "roofline": kernels[job.kernels[0][0]],
+        "roofline_step": roofline(bound, work, ms, pk, src, "whole step"),
+        "kernels": kernels,
+        "e2e": {"value": world * job.tokens / (e2e_ms * 1e-3),
+                "unit": "tokens/s" if w.kind != "mixed_decode" else "tokens/s (sequence x layer)",
+                "h2d_bytes_per_step": job.h2d, "d2h_bytes_per_step": job.d2h, "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+        "gpu_launches": job.launches_per_step * args.steps,
+        "timing": timing,
+    }
+    del job
+    torch.cuda.empty_cache()
+    return w, res
+
+
+def cpu_baseline(name, w):
+    """The oracle on a bounded sample of the workload, on this host's cores (about 10 s)."""
+    import oracle as O
+    if name == "hca_prefill_32k":
+        tps, secs, desc = oracle_hca_sample(w)
+    elif name == "csa_prefill_64k":
+        tps, secs, desc = oracle_csa_sample(w)
+    else:
+        job_o = OracleDecode(w, 4) if name == "csa_decode_1m" else OracleMixed(w, 8)
+        tps, secs, reps = oracle_repeat(job_o)
+        desc = f"{job_o.describe()}; the sample timed {reps} times over"
+    unit = "tokens/s (sequence x layer)" if w.kind == "mixed_decode" else "tokens/s"
+    return {"value": tps, "unit": unit, "cores": O.num_threads(), "kind": "oracle", "sample": desc, "seconds": secs}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="hca_prefill_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling a smaller case)")
     args = ap.parse_args()
-    w = WL.WORKLOADS[args.workload]
-    if args.T is not None:
-        import dataclasses
-        w = dataclasses.replace(w, T=args.T)
+    names = list(DEFAULT_WORKLOADS) if args.workload == "all" else [args.workload]
+    if args.T is not None and len(names) > 1:
+        ap.error("--T needs a single --workload")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    bad = check_world(args.gpus, world)
+    if bad is not None:
+        print(bad, file=sys.stderr)
+        return 2
 
     if args.impl == "reference":
-        return reference_arm(args, w, world, rank)
+        return reference_arm(args, WL.WORKLOADS[names[0]], world, rank)
 
     import torch
     import torch.distributed as dist
@@ -770,118 +1104,46 @@ def main():
                                 device_id=device)
     import compressed_sparse_kv_csa_b200 as C
 
-    job = WORKLOADS[args.workload](w, rank, torch, C, device)
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-
-    for _ in range(max(args.warmup, 3)):
-        job.step()
-    torch.cuda.synchronize()
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    props = torch.cuda.get_device_properties(local)
-    pci = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
-    with ClockSampler(local, pci) as clk:
-        start.record(stream)
-        for i in range(args.steps):
-            job.step(evs[i])
-        stop.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = start.elapsed_time(stop) / args.steps
-    kern_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    ms, kern_ms = max_over_ranks([ms, kern_ms], world, dist, device)
-
-    # end to end through the C ABI with host buffers
-    job.setup_e2e()
-    job.step_e2e()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        job.step_e2e()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    (e2e_ms,) = max_over_ranks([e2e_ms], world, dist, device)
-    if world > 1:
-        dist.barrier()
+    results = {}
+    for name in names:
+        results[name] = measure(name, args, world, rank, dist, device, torch, C)
 
     if rank == 0:
-        pk, src = peaks()
-        if hasattr(job, "bytes"):  # HBM-bound dominant kernel
-            achieved = job.bytes / (kern_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": job.kernel_name, "achieved": achieved, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": f"{src} HBM copy",
-                    "traffic": None, "bytes_per_launch": job.bytes, "launch_ms": kern_ms}
-        else:
-            achieved = job.flops / (kern_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "kernel": getattr(job, "kernel_name", "hybrid_attn_prefill"),
-                    "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / pk["bf16_tflops"], "peak_source": f"{src} dense bf16 burst",
-                    "traffic": None, "flops_per_launch": job.flops, "launch_ms": kern_ms}
-        cfg = {"workload": args.workload, "T": w.T, "c": w.c, "rope_dims": w.rope, "m": w.m, "H": w.H, "W": w.W,
-               "parallelism": f"replicas x{world}"}
-        if w.kind == "csa_decode":
-            cfg.update({"B": w.B, "n_comp_per_seq": (w.T + 1) // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
-                        "l2": "FP4 key scan (143 MB) and KV cache (1.2 GB) larger than L2"})
-        elif w.kind == "mixed_decode":
-            cfg = {"workload": args.workload, "B": w.B, "layers": list(w.extra["layers"]), "c": w.c,
-                   "rope_dims": w.rope, "H": w.H, "W": w.W, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
-                   "m_csa": w.extra["m_csa"], "m_hca": w.extra["m_hca"],
-                   "context": f"log-uniform [{w.extra['len_lo']}, {w.extra['len_hi']}]",
-                   "total_context_tokens": int(job.lens.sum()), "parallelism": f"replicas x{world}",
-                   "l2": "KV caches of the stack ({:.2f} GB) larger than L2".format(
-                       sum(L.comp.fp8.numel() + L.comp.rope.numel() * 2 + L.comp.scale.numel() * 4
-                           + (L.keys.codes.numel() + L.keys.scales.numel() if L.csa else 0)
-                           for L in job.layers) / 1e9)}
-        elif w.kind == "csa_prefill":
-            cfg.update({"n_comp": w.T // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
-                        "l2": "inputs larger than L2 (q alone is 4.3 GB)"})
-        else:
-            cfg.update({"n_comp": w.T // w.m, "l2": f"inputs larger than L2 (q alone is {w.T * w.H * w.c * 2 / 1e9:.1f} GB)"})
+        head_name = names[0]
+        w, head = results[head_name]
         line = {
             "metric": METRIC,
-            "value": world * job.tokens / (ms * 1e-3),
-            "unit": "tokens/s",
+            "value": head["value"],
+            "unit": head["unit"],
             "n_gpus": world,
             "steps": args.steps,
             "warmup": max(args.warmup, 3),
-            "ms_per_step": ms,
+            "ms_per_step": head["ms_per_step"],
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) inputs, bf16 grid / FP8 / FP4 caches, no trained weights)",
-            "config": cfg,
-            "roofline": roof,
-            "e2e": {"value": world * job.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": job.h2d, "d2h_bytes_per_step": job.d2h, "ms_per_step": e2e_ms},
-            "clocks": clk.summary(),
-            "gpu_launches": job.launches_per_step * args.steps,
+            "config": head["config"],
+            "roofline": head["roofline"],
+            "roofline_step": head["roofline_step"],
+            "kernels": head["kernels"],
+            "e2e": head["e2e"],
+            "clocks": head["clocks"],
+            "gpu_launches": head["gpu_launches"],
+            "timing": head["timing"],
         }
-        if not args.no_cpu_baseline and world == 1 and args.workload in ("hca_prefill_32k", "csa_decode_1m",
-                                                                          "mixed_decode_64"):
-            import oracle as O
-            if args.workload == "hca_prefill_32k":
-                tps, secs, desc = oracle_hca_sample(w)
-            else:
-                job_o = OracleDecode(w, 4) if args.workload == "csa_decode_1m" else OracleMixed(w, 8)
-                tps, secs, reps = oracle_repeat(job_o)
-                desc = f"{job_o.describe()}; the sample timed {reps} times over"
-            line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
-                                    "sample": desc, "seconds": secs}
+        if len(names) > 1:
+            line["workloads"] = {n: results[n][1] for n in names[1:]}
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(head_name, w)
+            for n in names[1:]:
+                line["workloads"][n]["cpu_baseline"] = cpu_baseline(n, results[n][0])
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
 
 
 def reference_arm(args, w, world, rank):
@@ -893,6 +1155,8 @@ def reference_arm(args, w, world, rank):
         job = OracleDecode(w, 1)
     elif w.kind == "mixed_decode":
         job = OracleMixed(w, 2)
+    elif w.kind == "csa_prefill":
+        job = OracleCsa(w, 1)
     else:
         job = OracleHca(w, 256)
     desc = job.describe()
@@ -918,4 +1182,4 @@ def reference_arm(args, w, world, rank):
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -221,17 +221,20 @@ def test_csa_decode_1m_full(C):
 
 def test_mixed_decode_64_stack_sampled(C):
     """The stacked decode workload as the bench builds it (64 sequences, layers HCA, CSA, HCA, CSA,
-    glue between layers), checked on the shortest, a median and the longest sequence.
+    glue between layers), checked in three parts.
 
-    The oracle runs the stack from the seeded inputs (layer outputs and next queries stored in
-    bf16, index queries in FP4, as on the GPU).  Each GPU layer is then checked on the oracle's
-    own inputs for that layer (oracle values fed to the GPU, never the reverse), so each check is
-    strict: top-k sets exact up to the 1e-4 tie band, attention outputs within 2e-2, glue as in
-    the glue parity test.  The bench's free-running GPU chain is checked for layer 0 (identical
-    inputs: strict); its later layers run on the GPU's own previous outputs, whose FP4 index
-    queries round some codes the other way than the oracle's, so the chain drifts from the
-    oracle's by more than the tolerance after two layers: there it is checked by top-k overlap
-    >= 75 % (an offset or wiring mistake gives almost none) and finite outputs."""
+    (a) Each GPU layer against the oracle on the oracle's own inputs for that layer (oracle
+        values fed to the GPU, never the reverse), on the shortest, a median and the longest
+        sequence: top-k sets exact up to the 1e-4 tie band, attention outputs within 2e-2, glue
+        as in the glue parity test.
+    (b) The bench's free-running chain, layer 0 (the oracle's inputs exactly): within 2e-2.
+    (c) The chain's composition: re-running every layer's calls on the chain's own stored inputs
+        reproduces its stored outputs bit for bit, so each layer of the chain is exactly the
+        layer function that (a) checks, wired to the right buffers, offsets and glue.
+    Later chain layers are not compared with the oracle's chain: their FP4 index queries round
+    values the GPU computes in fp32, and a rounding decision can flip for an input arbitrarily
+    close to a code boundary, so no tolerance on the inputs bounds the difference of the top-k
+    sets (their overlap is printed for information)."""
     import bench
     w = WL.WORKLOADS["mixed_decode_64"]
     job = bench.MixedDecode(w, 0, torch, C, torch.device("cuda", 0))
@@ -268,12 +271,14 @@ def test_mixed_decode_64_stack_sampled(C):
                 # GPU indexer on the oracle's index query (the same FP4 codes): strict
                 q4 = C.Fp4Rows(torch.from_numpy(qc).cuda(), torch.from_numpy(qs).cuda())
                 idx_g = C.indexer_topk(q4, dev(wt), L.keys, m, k, max_nvis=nv, q_pos=pos, key_off=off)
-                assert check_topk(idx_g.cpu().numpy(), idx_o, S, [nv], k) >= 0, (l, b)
-                # the free-running chain: overlap
+                check_topk(idx_g.cpu().numpy(), idx_o, S, [nv], k)  # asserts inside; returns the exact-set count
+                # the free-running chain: a valid list; its overlap with the oracle's is information only
                 ke = min(k, nv)
                 g = chain_idx[l][b]
                 assert np.all(g[ke:] == -1) and len(set(g[:ke].tolist())) == ke
-                assert len(set(g[:ke].tolist()) & set(idx_o[0, :ke].tolist())) >= 0.75 * ke, (l, b)
+                assert np.all((g[:ke] >= 0) & (g[:ke] < nv))
+                print(f"chain layer {l} seq {b}: top-k overlap with the oracle's chain "
+                      f"{len(set(g[:ke].tolist()) & set(idx_o[0, :ke].tolist())) / ke:.3f}")
                 sel = np.sort(idx_o[0, :ke])
                 f8, rb, sc = O.quant_kv(WL.draw(w, "KV", 0, nv, layer=l, seq=b)[sel])
                 comp = O.dequant_kv(f8, rb, sc)
@@ -289,7 +294,6 @@ def test_mixed_decode_64_stack_sampled(C):
                 o_g = C.hybrid_attn_decode(q_bf, L.comp, off, pos, win_b, wl1, dev(sink), 1.0, m, W, max_nvis=nv)
             err = row_rel_err(host(o_g), o_ref)
             assert err.max() < 2e-2, (l, b, t, err.max())
-            assert np.isfinite(chain_o[l][b]).all()
             if l == 0:  # the free-running chain's first layer has exactly the oracle's inputs
                 assert row_rel_err(chain_o[l][b:b + 1], o_ref).max() < 2e-2
             if l + 1 < len(job.layers):
@@ -303,4 +307,23 @@ def test_mixed_decode_64_stack_sampled(C):
                 if qI_g is not None:
                     check_fp4_near(qI_g.codes.cpu().numpy(), qI_g.scales.cpu().numpy(), zi)
                 q = O.bf16_value(O.bf16_bits(qn)).reshape(1, H, c).astype(np.float64)
+    assert C.csa_device_error() == 0
+
+    # (c) composition: each layer's calls re-run on the chain's stored inputs give its stored outputs
+    q_in = job.q0
+    for l, L in enumerate(job.layers):
+        if L.csa:
+            idx_re = C.indexer_topk(L.qI, L.wI, L.keys, L.m, k, max_nvis=L.max_nv, q_pos=job.pos, key_off=L.off)
+            assert torch.equal(idx_re, L.idx), l
+        o_re = C.hybrid_attn_decode(q_in, L.comp, L.off, job.pos, L.win, job.win_len, L.sink, 1.0, L.m, W,
+                                    max_nvis=L.max_nv, idx=L.idx if L.csa else None)
+        assert torch.equal(o_re, L.o), l
+        if l + 1 < len(job.layers):
+            nxt = job.layers[l + 1]
+            qn_re, qI_re = C.csa_decode_glue(L.o, L.P, L.Rm)
+            assert torch.equal(qn_re, L.q_next), l
+            if nxt.csa:
+                assert torch.equal(qI_re.codes, nxt.qI.codes) and torch.equal(qI_re.scales, nxt.qI.scales), l
+            q_in = L.q_next
+    torch.cuda.synchronize()
     assert C.csa_device_error() == 0

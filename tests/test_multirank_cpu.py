@@ -60,3 +60,48 @@ def test_single_rank_is_identity():
     assert bench.max_over_ranks([3.0, 4.0], 1, None, None) == [3.0, 4.0]
     assert bench.rank_sequences(4, 0) == [0, 1, 2, 3]
     assert bench.rank_sequences(4, 2) == [8, 9, 10, 11]
+
+
+def _world_worker(rank: int, world: int, port: int, q):
+    """Each rank runs bench.py's entry check with its launcher's WORLD_SIZE, as torchrun sets it."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        ok = bench.check_world(world, world)
+        refused = bench.check_world(1, world)
+        dist.barrier()
+        q.put((rank, ok, refused))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_refuses_gpus_that_do_not_match_the_ranks():
+    """`bench.py --gpus N` runs only when the launcher started N ranks (one per GPU): two gloo
+    ranks accept --gpus 2 and refuse --gpus 1; a single process refuses --gpus 8."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_world_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=120) for _ in range(2)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, ok, refused in res:
+        assert ok is None and refused is not None and "WORLD_SIZE=2" in refused
+    import bench
+    assert bench.check_world(1, 1) is None
+    assert "WORLD_SIZE=1" in bench.check_world(8, 1)
+
+
+def test_bench_main_exits_nonzero_on_mismatch():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "4", "--impl", "reference"],
+                         capture_output=True, text=True, timeout=120, cwd=root, env=env)
+    assert out.returncode == 2 and "--gpus 4 but WORLD_SIZE=1" in out.stderr
