@@ -88,6 +88,9 @@ def lib():
             L.orc_quant_kv.argtypes = [_f32p, _i64, _int, _int, _u8p, _u16p, _f32p]
             L.orc_dequant_kv.argtypes = [_u8p, _u16p, _f32p, _i64, _int, _int, _f64p]
             L.orc_decode_glue.argtypes = [_f64p, _f64p, _f64p, _i64, _int, _int, _f64p, _f64p]
+            L.orc_rmsnorm.argtypes = [_f64p, _f64p, _i64, _int, ctypes.c_double, _f64p]
+            L.orc_rope.argtypes = [_f64p, _i64p, _i64, _int, _int, ctypes.c_double, _f64p]
+            L.orc_hadamard.argtypes = [_f64p, _i64, _int, _f64p]
             L.orc_num_threads.restype = ctypes.c_int
             _lib = L
     return _lib
@@ -361,3 +364,38 @@ def decode_glue(o, P, Rm):
     zi = np.empty((R, d), np.float64)
     lib().orc_decode_glue(_p(o, _f64p), _p(P, _f64p), _p(Rm, _f64p), R, c, d, _p(qn, _f64p), _p(zi, _f64p))
     return qn, zi
+
+
+# ----------------------------------------------------------------------------------------
+# layer fidelity: RMSNorm, rotary embedding, Hadamard rotation
+# ----------------------------------------------------------------------------------------
+
+def rmsnorm(x, g, eps: float):
+    """Rows x [n, d] -> x / sqrt(mean(x^2) + eps) * g ([notes] Sec. 2.3 Compressor listing)."""
+    x, g = _f64(x), _f64(g)
+    n, d = x.shape
+    out = np.empty_like(x)
+    lib().orc_rmsnorm(_p(x, _f64p), _p(g, _f64p), n, d, float(eps), _p(out, _f64p))
+    return out
+
+
+def rope(x, pos, rd: int, base: float = 10000.0):
+    """Rotary embedding of the last rd channels of rows x [n, d] at positions pos [n]
+    ([notes] Sec. 2.3 Indexer listing, apply_rotary_emb(q[..., -rd:], freqs_cis))."""
+    x = _f64(x)
+    n, d = x.shape
+    pos = np.ascontiguousarray(pos, np.int64)
+    out = np.empty_like(x)
+    lib().orc_rope(_p(x, _f64p), _p(pos, _i64p), n, d, int(rd), float(base), _p(out, _f64p))
+    return out
+
+
+def hadamard(x):
+    """Rows x [n, d] (d a power of two) -> x H / sqrt(d) with the Sylvester Hadamard matrix
+    ([notes] Sec. 2.3 Indexer listing, rotate_activation)."""
+    x = _f64(x)
+    n, d = x.shape
+    assert d & (d - 1) == 0
+    out = np.empty_like(x)
+    lib().orc_hadamard(_p(x, _f64p), n, d, _p(out, _f64p))
+    return out

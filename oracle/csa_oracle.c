@@ -460,3 +460,65 @@ void orc_decode_glue(const double *o, const double *P, const double *Rm, int64_t
         for (int i = 0; i < d; i++) zi[r * d + i] *= f;
     }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Layer fidelity: RMSNorm of entries, rotary embedding of the last dims, Hadamard rotation      */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * RMSNorm of rows, [notes] Sec. 2.3 Compressor listing (self.norm = RMSNorm(head_dim, norm_eps),
+ * applied to the compressed entries) with the normalisation written out in the mHC listing
+ * (rsqrt(mean(x^2) + eps)):  out[r, j] = x[r, j] / sqrt(mean_j x[r, j]^2 + eps) * g[j].
+ */
+void orc_rmsnorm(const double *x, const double *g, int64_t n, int d, double eps, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; r++) {
+        double ss = 0.0;
+        for (int j = 0; j < d; j++) ss += x[r * d + j] * x[r * d + j];
+        const double f = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; j++) out[r * d + j] = x[r * d + j] * f * g[j];
+    }
+}
+
+/*
+ * Rotary embedding of the last rd channels of each row, [notes] Sec. 2.3 Indexer listing
+ * (apply_rotary_emb(q[..., -rd:], freqs_cis)): inside that slice the channel pairs (2i, 2i+1)
+ * rotate by the angle a = pos[r] * base^(-2i/rd):
+ *   y[2i] = x[2i] cos a - x[2i+1] sin a,   y[2i+1] = x[2i] sin a + x[2i+1] cos a.
+ * The first d - rd channels are copied.
+ */
+void orc_rope(const double *x, const int64_t *pos, int64_t n, int d, int rd, double base, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; r++) {
+        const double *xr = x + r * d;
+        double *yr = out + r * d;
+        for (int j = 0; j < d - rd; j++) yr[j] = xr[j];
+        for (int i = 0; i < rd / 2; i++) {
+            const double a = (double)pos[r] * pow(base, -2.0 * i / rd);
+            const double x0 = xr[d - rd + 2 * i], x1 = xr[d - rd + 2 * i + 1];
+            yr[d - rd + 2 * i] = x0 * cos(a) - x1 * sin(a);
+            yr[d - rd + 2 * i + 1] = x0 * sin(a) + x1 * cos(a);
+        }
+    }
+}
+
+/*
+ * Hadamard rotation of rows of d = 2^p channels, [notes] Sec. 2.3 Indexer listing
+ * (rotate_activation before the FP4 quantisation of the index queries and keys):
+ *   out[r, i] = sum_j x[r, j] H[j, i] / sqrt(d),   H[j, i] = (-1)^popcount(i & j)
+ * (the Sylvester matrix: H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]), written as the plain sum.
+ */
+void orc_hadamard(const double *x, int64_t n, int d, double *out)
+{
+    const double s = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; r++) {
+        for (int i = 0; i < d; i++) {
+            double acc = 0.0;
+            for (int j = 0; j < d; j++) acc += (__builtin_popcount((unsigned)(i & j)) & 1) ? -x[r * d + j] : x[r * d + j];
+            out[r * d + i] = acc * s;
+        }
+    }
+}

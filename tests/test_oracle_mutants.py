@@ -86,6 +86,17 @@ C_MUTANTS = [
     ("glue_drop_sqrt_c", "1.0 / sqrt(ss / c) / sqrt((double)c)", "1.0 / sqrt(ss / c)"),
     ("glue_transposed_p", "P[(int64_t)i * c + j]", "P[(int64_t)j * c + i]"),
     ("glue_index_query_norm_by_c", "1.0 / sqrt(ss / d) : 0.0", "1.0 / sqrt(ss / c) : 0.0"),
+    # layer fidelity (Sec. 2.3 Compressor and Indexer listings)
+    ("rmsnorm_drops_eps", "const double f = 1.0 / sqrt(ss / d + eps);", "const double f = 1.0 / sqrt(ss / d);"),
+    ("rmsnorm_sum_not_mean", "const double f = 1.0 / sqrt(ss / d + eps);", "const double f = 1.0 / sqrt(ss + eps);"),
+    ("rmsnorm_drops_gain", "out[r * d + j] = x[r * d + j] * f * g[j];", "out[r * d + j] = x[r * d + j] * f;"),
+    ("rope_clockwise", "yr[d - rd + 2 * i] = x0 * cos(a) - x1 * sin(a);", "yr[d - rd + 2 * i] = x0 * cos(a) + x1 * sin(a);"),
+    ("rope_exponent_sign", "pow(base, -2.0 * i / rd)", "pow(base, 2.0 * i / rd)"),
+    ("rope_exponent_not_halved", "pow(base, -2.0 * i / rd)", "pow(base, -1.0 * i / rd)"),
+    ("rope_first_dims", "const double x0 = xr[d - rd + 2 * i], x1 = xr[d - rd + 2 * i + 1];",
+     "const double x0 = xr[2 * i], x1 = xr[2 * i + 1];"),
+    ("hadamard_not_normalised", "out[r * d + i] = acc * s;", "out[r * d + i] = acc;"),
+    ("hadamard_wrong_sign_rule", "(__builtin_popcount((unsigned)(i & j)) & 1)", "(__builtin_popcount((unsigned)(i | j)) & 1)"),
 ]
 
 # (name, old text, new text) on the Python half: key lists and visibility.

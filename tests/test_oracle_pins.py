@@ -524,3 +524,77 @@ def test_glue_normalisation_identity_and_symmetry():
     np.testing.assert_allclose(qa, y / np.sqrt((y ** 2).mean(1, keepdims=True)) / np.sqrt(c), rtol=1e-12)
     z0, _ = O.decode_glue(np.zeros((2, c)), P, Rm)
     assert np.all(z0 == 0)
+
+
+# ---------------------------------------------------------------------------------------------
+# layer fidelity: RMSNorm of entries, rotary embedding, Hadamard rotation
+# ([notes] Sec. 2.3 Compressor and Indexer listings)
+# ---------------------------------------------------------------------------------------------
+
+def test_rmsnorm_unit_rms_scale_invariance_and_gain():
+    g = np.random.default_rng(30)
+    x = g.standard_normal((6, 512))
+    y = O.rmsnorm(x, np.ones(512), 0.0)
+    np.testing.assert_allclose(np.sqrt((y ** 2).mean(1)), 1.0, rtol=1e-12)       # unit RMS per row
+    np.testing.assert_allclose(O.rmsnorm(7.5 * x, np.ones(512), 0.0), y, rtol=1e-12)  # scale invariance
+    gain = g.standard_normal(512)
+    np.testing.assert_allclose(O.rmsnorm(x, gain, 0.0), y * gain, rtol=1e-12)   # gain per channel
+    # hand example: [3, 4] has mean square 12.5; with eps = 0.5 the divisor is sqrt(13)
+    np.testing.assert_allclose(O.rmsnorm(np.array([[3.0, 4.0]]), np.ones(2), 0.5), [[3 / np.sqrt(13), 4 / np.sqrt(13)]])
+    assert np.all(O.rmsnorm(np.zeros((1, 8)), np.ones(8), 1e-6) == 0.0)
+
+
+def test_rope_identity_norms_and_untouched_leading_channels():
+    g = np.random.default_rng(31)
+    x = g.standard_normal((4, 512))
+    y = O.rope(x, np.zeros(4, np.int64), 64)
+    np.testing.assert_array_equal(y, x)                                    # position 0: identity
+    y = O.rope(x, np.array([1, 77, 4096, 1048576]), 64)
+    np.testing.assert_array_equal(y[:, :448], x[:, :448])                  # only the last 64 rotate
+    pairs_x = x[:, 448:].reshape(4, 32, 2)
+    pairs_y = y[:, 448:].reshape(4, 32, 2)
+    np.testing.assert_allclose(np.linalg.norm(pairs_y, axis=-1), np.linalg.norm(pairs_x, axis=-1), rtol=1e-12)
+
+
+def test_rope_frequencies_and_rotation_direction():
+    """Unit vectors (1, 0) in every pair at position 1 come out at the angle of the pair's
+    frequency base^(-2i/rd), counter-clockwise: (cos f, sin f)."""
+    rd, base = 64, 10000.0
+    x = np.tile([1.0, 0.0], rd // 2)[None, :]
+    y = O.rope(x, np.array([1]), rd, base).reshape(rd // 2, 2)
+    f = base ** (-np.arange(rd // 2) * 2.0 / rd)
+    np.testing.assert_allclose(np.arctan2(y[:, 1], y[:, 0]), f, rtol=1e-12)
+    np.testing.assert_allclose(y[0], [np.cos(1.0), np.sin(1.0)], rtol=1e-14)
+
+
+def test_rope_composes_and_keeps_relative_positions():
+    g = np.random.default_rng(32)
+    q, k = g.standard_normal((2, 128))
+    a, b, s = 300, 41, 9000
+    two = O.rope(O.rope(q[None], np.array([a]), 64), np.array([b]), 64)
+    np.testing.assert_allclose(two, O.rope(q[None], np.array([a + b]), 64), atol=1e-9)
+    d1 = O.rope(q[None], np.array([a]), 64) @ O.rope(k[None], np.array([b]), 64).T
+    d2 = O.rope(q[None], np.array([a + s]), 64) @ O.rope(k[None], np.array([b + s]), 64).T
+    np.testing.assert_allclose(d1, d2, rtol=1e-9)
+
+
+def test_hadamard_matches_the_library_matrix_and_is_an_involution():
+    import scipy.linalg
+    g = np.random.default_rng(33)
+    for d in (32, 128, 512):
+        x = g.standard_normal((3, d))
+        y = O.hadamard(x)
+        np.testing.assert_allclose(y, x @ scipy.linalg.hadamard(d) / np.sqrt(d), atol=1e-12)
+        np.testing.assert_allclose(O.hadamard(y), x, atol=1e-12)          # normalised Sylvester: H H = I
+        np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    e0 = np.zeros((1, 128))
+    e0[0, 0] = 1.0
+    np.testing.assert_allclose(O.hadamard(e0), np.full((1, 128), 1 / np.sqrt(128)), rtol=1e-14)
+
+
+def test_hadamard_recursive_definition():
+    """H_2n = [[H_n, H_n], [H_n, -H_n]] built recursively, column by column."""
+    H = np.array([[1.0]])
+    while H.shape[0] < 64:
+        H = np.block([[H, H], [H, -H]])
+    np.testing.assert_allclose(O.hadamard(np.eye(64)), H / 8.0, atol=1e-14)
