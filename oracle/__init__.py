@@ -399,3 +399,41 @@ def hadamard(x):
     out = np.empty_like(x)
     lib().orc_hadamard(_p(x, _f64p), n, d, _p(out, _f64p))
     return out
+
+
+# ----------------------------------------------------------------------------------------
+# decode append path: the state cache of one sequence
+# ----------------------------------------------------------------------------------------
+
+class AppendState:
+    """The decode-time state of one layer of one sequence ([qa] Question 5: the compression tail
+    tokens are kept in a fixed state cache; [notes] Sec. 2.3 Compressor listing: an entry is
+    emitted once its block is complete).  append(t, rows) takes token t's compressor rows --
+    (Ca, Cb, Za, Zb) for CSA, (C, Z) for HCA, each [c] -- keeps the last L tokens (L = 2m for the
+    overlapped CSA compression, m for HCA) and, when token t completes block e = (t+1)/m - 1,
+    returns entry e pooled by the same compression as the prefill over exactly the tokens that
+    entry reads; otherwise None.  Tokens must arrive in order from 0."""
+
+    def __init__(self, overlap: bool, m: int, B):
+        self.overlap, self.m, self.B = overlap, m, np.asarray(B, np.float64)
+        self.L = 2 * m if overlap else m
+        self.ring = {}
+        self.next_t = 0
+
+    def append(self, t: int, rows):
+        assert t == self.next_t, "tokens arrive in order"
+        self.next_t += 1
+        self.ring[t] = [np.asarray(r, np.float64) for r in rows]
+        self.ring.pop(t - self.L, None)
+        m = self.m
+        if (t + 1) % m:
+            return None
+        e = (t + 1) // m - 1
+        if self.overlap:
+            first = max(0, (e - 1) * m)           # previous block (absent for entry 0), then this one
+            toks = range(first, t + 1)
+            Ca, Cb, Za, Zb = (np.stack([self.ring[p][i] for p in toks]) for i in range(4))
+            return csa_compress(Ca, Cb, Za, Zb, self.B, m)[-1]
+        toks = range(e * m, t + 1)
+        C, Z = (np.stack([self.ring[p][i] for p in toks]) for i in range(2))
+        return hca_compress(C, Z, self.B, m)[0]

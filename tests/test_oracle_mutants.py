@@ -117,6 +117,9 @@ PY_MUTANTS = [
     ("decode_hca_visibility", "s = np.arange(int(n_vis(int(pos[b]), m)), dtype=np.int64)",
      "s = np.arange(int(pos[b]) // m, dtype=np.int64)"),
     ("decode_csa_keeps_padding", "            s = r[r >= 0]\n", "            s = r\n"),
+    ("append_emits_one_token_late", "        if (t + 1) % m:\n            return None", "        if t % m or t == 0:\n            return None"),
+    ("append_overlap_skips_previous_block", "            first = max(0, (e - 1) * m)", "            first = e * m"),
+    ("append_ring_too_short", "        self.L = 2 * m if overlap else m", "        self.L = m"),
     ("bf16_vector_ties_away", "r = ((u + 0x7FFF + lsb) >> 16)", "r = ((u + 0x8000) >> 16)"),
 ]
 
@@ -147,7 +150,10 @@ def _pin_cases():
         params = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
         if params:
             (argname, values), = [m.args for m in params]
-            cases += [(f"{name}[{v}]", fn, {argname: v}) for v in values]
+            names = [a.strip() for a in argname.split(",")]
+            for v in values:
+                kw = dict(zip(names, v)) if len(names) > 1 else {argname: v}
+                cases.append((f"{name}[{v}]", fn, kw))
         else:
             cases.append((name, fn, {}))
         needed = set(inspect.signature(fn).parameters)

@@ -598,3 +598,29 @@ def test_hadamard_recursive_definition():
     while H.shape[0] < 64:
         H = np.block([[H, H], [H, -H]])
     np.testing.assert_allclose(O.hadamard(np.eye(64)), H / 8.0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------------
+# decode append path ([qa] Question 5 state cache; [notes] Sec. 2.3 Compressor decode branch)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("overlap,m,T", [(True, 4, 61), (False, 16, 70), (True, 1, 9), (False, 1, 5)])
+def test_append_one_token_at_a_time_equals_the_prefill_compression(overlap, m, T):
+    """Entries emitted by the state cache as tokens arrive one by one are bit for bit the prefill
+    compression's entries, in order, one per completed block (a trailing partial block emits
+    nothing)."""
+    g = np.random.default_rng(40 + m)
+    c = 16
+    n_arr = 4 if overlap else 2
+    X = [g.standard_normal((T, c)) for _ in range(n_arr)]
+    B = 0.1 * g.standard_normal((2 * m if overlap else m, c))
+    st = O.AppendState(overlap, m, B)
+    got = []
+    for t in range(T):
+        e = st.append(t, [x[t] for x in X])
+        assert (e is not None) == ((t + 1) % m == 0)
+        if e is not None:
+            got.append(e)
+    ref = O.csa_compress(*X, B, m) if overlap else O.hca_compress(*X, B, m)
+    assert len(got) == T // m
+    np.testing.assert_array_equal(np.stack(got), ref)
