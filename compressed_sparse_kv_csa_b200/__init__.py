@@ -28,10 +28,11 @@ CSA_F32 = 0
 CSA_BF16 = 1
 CSA_FP4 = 2
 
-EXPORTED = ("csa_compress", "hca_compress", "csa_quantize_kv", "csa_quantize_fp4",
+EXPORTED = ("csa_compress", "hca_compress", "csa_quantize_kv", "csa_quantize_fp4", "csa_prep_rows",
+            "csa_window_append", "csa_compress_append", "indexer_topk_paged", "hybrid_attn_decode_paged",
             "indexer_topk_workspace_size", "indexer_topk", "hybrid_attn_prefill",
             "hybrid_attn_decode_workspace_size", "hybrid_attn_decode", "csa_device_error",
-            "csa_status_string", "csa_abi_version")
+            "csa_status_string", "csa_abi_version", "csa_last_path", "csa_set_wait_limit_ns")
 
 
 class CsaError(RuntimeError):
@@ -62,6 +63,15 @@ def _load():
         "hca_compress": ([vp, vp, vp, i64, i32, i32, i32, vp, i32, P_kv, vp], ctypes.c_int),
         "csa_quantize_kv": ([vp, i32, i64, i32, i32, P_kv, vp], ctypes.c_int),
         "csa_quantize_fp4": ([vp, i32, i64, i32, P_f4, vp], ctypes.c_int),
+        "indexer_topk_paged": ([vp, vp, vp, vp, i64, i32, i32, i32, i32, i64, vp, i32, i32, vp, vp, vp, sz, vp],
+                               ctypes.c_int),
+        "hybrid_attn_decode_paged": ([vp, P_kv, vp, i32, i32, vp, P_kv, vp, vp, i32, vp, f32, i32, i32, i32, i32, i32,
+                                      i64, vp, vp, vp, sz, vp], ctypes.c_int),
+        "csa_window_append": ([vp, i32, i64, i32, vp, i32, P_kv, vp], ctypes.c_int),
+        "csa_compress_append": ([i32, i64, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, P_kv, P_f4, vp, i32,
+                                 i32, vp, vp], ctypes.c_int),
+        "csa_prep_rows": ([vp, i32, i64, i32, vp, f32, i32, vp, ctypes.c_double, i32, vp, i32, P_kv, P_f4, vp],
+                          ctypes.c_int),
         "indexer_topk_workspace_size": ([i64, i64, i32], sz),
         "indexer_topk": ([vp, vp, vp, i32, vp, vp, i64, i64, i32, i32, i32, i32, i64, vp, vp, vp, sz, vp],
                          ctypes.c_int),
@@ -77,6 +87,8 @@ def _load():
         "csa_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
         "csa_status_string": ([i32], ctypes.c_char_p),
         "csa_abi_version": ([], i32),
+        "csa_last_path": ([], i32),
+        "csa_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -218,6 +230,50 @@ def csa_quantize_fp4(x, out: Fp4Rows, stream=None):
     return out
 
 
+def csa_window_append(x, pos, W: int, win: KvRows, stream=None):
+    """Quantise the new tokens' raw KV rows x [B, c] into the window rings (row b*W + pos[b] % W)."""
+    B, c = x.shape
+    _check("csa_window_append", _lib.csa_window_append(_ptr(x), _dtype_code(x), B, c, _ptr(pos), int(W),
+                                                       ctypes.byref(win._c()), _stream(stream)))
+    return win
+
+
+def csa_compress_append(rows, tail, B_bias, m: int, pos, out_kv: KvRows | None = None,
+                        out_fp4: Fp4Rows | None = None, pages=None, page_rows: int = 0, comp_off=None, stream=None):
+    """Append the new tokens' compressor rows to the tail rings and emit the entries whose block
+    they complete.  rows = (Ca, Cb, Za, Zb) for CSA or (C, Z) for HCA, each [B, c]; tail = the
+    matching rings [B, L, c] (L = 2m or m).  Entries go to out_kv or out_fp4 through the page table
+    pages [B, max_pages] (page_rows entries per page) or at comp_off[b] + e."""
+    overlap = len(rows) == 4
+    B, c = rows[0].shape
+    r = list(rows) + [None] * (4 - len(rows))
+    t = list(tail) + [None] * (4 - len(tail))
+    if not overlap:  # HCA: C -> Ca, Z -> Za
+        r = [rows[0], None, rows[1], None]
+        t = [tail[0], None, tail[1], None]
+    st = _lib.csa_compress_append(1 if overlap else 0, B, _ptr(pos), c, int(m), _dtype_code(rows[0]),
+                                  *(_ptr(x) for x in r), *(_ptr(x) for x in t), _ptr(B_bias),
+                                  ctypes.byref(out_kv._c()) if out_kv is not None else None,
+                                  ctypes.byref(out_fp4._c()) if out_fp4 is not None else None,
+                                  _ptr(pages), pages.shape[1] if pages is not None else 0, int(page_rows),
+                                  _ptr(comp_off), _stream(stream))
+    _check("csa_compress_append", st)
+
+
+def csa_prep_rows(x, g=None, eps: float = 1e-6, rd: int = 0, pos=None, base: float = 10000.0,
+                  hadamard: bool = False, out=None, out_kv: KvRows | None = None, out_fp4: Fp4Rows | None = None,
+                  stream=None):
+    """RMSNorm (when g is given), rotary embedding of the last rd channels at positions pos, Hadamard
+    rotation (when asked) of the rows x [n, d], written to any of out / out_kv / out_fp4."""
+    n, d = x.shape
+    st = _lib.csa_prep_rows(_ptr(x), _dtype_code(x), n, d, _ptr(g), float(eps), int(rd), _ptr(pos), float(base),
+                            1 if hadamard else 0, _ptr(out), _dtype_code(out) if out is not None else 0,
+                            ctypes.byref(out_kv._c()) if out_kv is not None else None,
+                            ctypes.byref(out_fp4._c()) if out_fp4 is not None else None, _stream(stream))
+    _check("csa_prep_rows", st)
+    return out
+
+
 def indexer_topk_workspace_size(Nq: int, max_nvis: int, k: int) -> int:
     return int(_lib.indexer_topk_workspace_size(Nq, max_nvis, k))
 
@@ -314,6 +370,42 @@ def hybrid_attn_decode(q, comp: KvRows, comp_off, pos, win: KvRows, win_len, sin
     return o
 
 
+def hybrid_attn_decode_paged(q, comp: KvRows, pages, page_rows: int, pos, win: KvRows, win_len, sink, scale: float,
+                             m: int, W: int, max_nvis: int, idx=None, o=None, lse=None, workspace=None, stream=None):
+    """hybrid_attn_decode over a paged compressed cache: pages [B, max_pages] int32 page ids of
+    page_rows entries each."""
+    B, H, c = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    k = idx.shape[1] if idx is not None else 0
+    need = hybrid_attn_decode_workspace_size(B, H, c, k, W, max_nvis, idx is not None)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
+    st = _lib.hybrid_attn_decode_paged(_ptr(q), ctypes.byref(comp._c()), _ptr(pages), pages.shape[1], int(page_rows),
+                                       _ptr(pos), ctypes.byref(win._c()), _ptr(win_len), _ptr(idx), k, _ptr(sink),
+                                       float(scale), B, H, c, m, W, max_nvis, _ptr(o), _ptr(lse), _ptr(workspace),
+                                       workspace.numel(), _stream(stream))
+    _check("hybrid_attn_decode_paged", st)
+    return o
+
+
+def indexer_topk_paged(q: Fp4Rows, w, keys: Fp4Rows, m: int, k: int, max_nvis: int, pages, page_rows: int,
+                       q_pos=None, idx_out=None, score_out=None, workspace=None, stream=None):
+    """FP4 indexer top-k over paged index keys: pages [Nq, max_pages] int32 page ids of page_rows
+    keys each.  Returns idx_out [Nq, k] int32."""
+    Nq, H_I = w.shape
+    if idx_out is None:
+        idx_out = torch.empty((Nq, k), dtype=torch.int32, device=q.codes.device)
+    need = indexer_topk_workspace_size(Nq, max_nvis, k)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.codes.device)
+    st = _lib.indexer_topk_paged(ctypes.byref(q._c()), _ptr(w), ctypes.byref(keys._c()), _ptr(q_pos), Nq, H_I, q.d, m,
+                                 k, max_nvis, _ptr(pages), pages.shape[1], int(page_rows), _ptr(idx_out),
+                                 _ptr(score_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("indexer_topk_paged", st)
+    return idx_out
+
+
 def csa_decode_glue(o, P, Rm=None, q_next=None, qI: Fp4Rows | None = None, stream=None):
     """Inter-layer projection of a decode stack: q_next = bf16(RMS-normalised P o / sqrt(c)) and,
     when Rm is given, qI = FP4(RMS-normalised Rm o).  o is [..., c] bf16 (rows = sequences x
@@ -339,3 +431,25 @@ def csa_device_error(stream=None) -> int:
 
 def csa_abi_version() -> int:
     return int(_lib.csa_abi_version())
+
+
+# kernel paths reported by csa_last_path (include/csa.h)
+CSA_PATH_NONE = 0
+CSA_PATH_INDEXER_FP4_TC = 1
+CSA_PATH_INDEXER_BF16_TC = 2
+CSA_PATH_INDEXER_GENERIC = 3
+CSA_PATH_PREFILL_TC = 4
+CSA_PATH_PREFILL_GENERIC = 5
+CSA_PATH_DECODE_TC = 6
+CSA_PATH_DECODE_GENERIC = 7
+CSA_PATH_PREFILL_PAIR_TC = 8
+
+
+def csa_set_wait_limit_ns(ns: int) -> int:
+    """Limit of the decode tensor-core kernel's bounded waits for later calls (0 = 2 s default)."""
+    return int(_lib.csa_set_wait_limit_ns(int(ns)))
+
+
+def csa_last_path() -> int:
+    """The kernel path that served this host thread's last indexer / attention call."""
+    return int(_lib.csa_last_path())

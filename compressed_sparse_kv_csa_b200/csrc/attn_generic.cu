@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(NWARP * 32) prefill_generic_kernel(PrefillArgs
                     int64_t s;
                     if (a.idx) {
                         s = a.idx[t * a.k + (j - n_win)];
-                        if (s >= a.n_comp) {
+                        if (s >= a.n_comp || s >= (t + 1) / a.m) { // missing, or not yet visible to t
                             if (ch == 0) flag_error(a.err, CSA_DEVERR_INDEX);
                             s = -1;
                         }
@@ -199,7 +199,9 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
     const int64_t n_keys = n_win + n_cmp;
     const int64_t c0 = (int64_t)chunk * a.chunk;
     const int64_t c1 = (c0 + a.chunk) < n_keys ? (c0 + a.chunk) : n_keys;
-    const int64_t cbase = a.comp_off[b];
+    const int64_t cbase = a.pages ? 0 : a.comp_off[b];
+    int64_t n_vis = (a.pos[b] + 1) / a.m; // entries of this sequence the new token may see
+    if (n_vis > a.max_nvis) n_vis = a.max_nvis;
 
     // gather key rows j0 .. j0+KT-1 of this sequence's list (dequantised to fp32) into the tile
     auto stage = [&](int64_t j0) {
@@ -214,8 +216,8 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
             } else if (j < c1) {        // compressed entry
                 const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
                 if (s >= 0) {
-                    const int64_t row = cbase + s;
-                    if (row >= 0 && row < a.comp.n) {
+                    const int64_t row = paged_row(a.pages, a.max_pages, a.page_rows, b, s, cbase);
+                    if (s < n_vis && row >= 0 && row < a.comp.n) {
                         v = kv_row4(a.comp, row, ch);
                         ok = 1;
                     } else if (ch == 0) {
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(NWARP * 32) decode_partial_kernel(DecodeArgs a
 // The per-chunk weights e^{m_j - m} / denominator are computed once into shared memory.
 constexpr int kMaxMergeChunks = 1024;
 
-__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a)
+__global__ void __launch_bounds__(128) attn_merge_kernel(DecodeArgs a)
 {
     __shared__ float fac[kMaxMergeChunks], lsum[kMaxMergeChunks];
     __shared__ float red[8];
@@ -351,7 +353,7 @@ cudaError_t decode_launch(const DecodeArgs &a, cudaStream_t st)
     kern<<<dim3((unsigned)a.n_chunks, (unsigned)a.B), NWARP * 32, smem, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<(unsigned)(a.B * a.H), 128, 0, st>>>(a);
+    attn_merge_kernel<<<(unsigned)(a.B * a.H), 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -368,7 +370,7 @@ void decode_plan(int B, int H, int c, int max_keys, int *n_chunks, int *chunk)
 {
     (void)H;
     (void)c;
-    const int target = 2 * 148;
+    const int target = 2 * device_sms(); // two CTAs per SM over the batch
     int nc = (target + B - 1) / (B > 0 ? B : 1);
     const int max_nc = (max_keys + KT - 1) / KT;
     if (nc > max_nc) nc = max_nc;
@@ -384,7 +386,7 @@ void decode_plan(int B, int H, int c, int max_keys, int *n_chunks, int *chunk)
 cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st)
 {
     if (a.n_chunks > kMaxMergeChunks) return cudaErrorInvalidValue;
-    decode_merge_kernel<<<(unsigned)(a.B * a.H), 128, 0, st>>>(a);
+    attn_merge_kernel<<<(unsigned)(a.B * a.H), 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 

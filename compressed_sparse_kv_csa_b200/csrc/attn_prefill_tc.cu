@@ -85,7 +85,7 @@ __device__ __forceinline__ const uint16_t *key_row(const PrefillArgs &a, int64_t
     if (slot >= n_cmp) return nullptr;
     const int64_t s = a.idx ? (int64_t)a.idx[t * a.k + slot] : slot;
     if (s < 0) return nullptr;
-    if (s >= a.n_comp) {
+    if (s >= a.n_comp || s >= (t + 1) / a.m) { // missing, or not yet visible to t
         if (report) flag_error(a.err, CSA_DEVERR_INDEX);
         return nullptr;
     }
@@ -133,7 +133,7 @@ __device__ __forceinline__ int32_t gather_row(const PrefillArgs &a, int64_t t, i
     const int64_t slot = (int64_t)(i - 1) * kKT + j;
     if (slot >= n_cmp) return -1;
     const int32_t s = a.idx[t * a.k + slot];
-    if (s >= a.n_comp) {
+    if (s >= a.n_comp || s >= (t + 1) / a.m) { // missing, or not yet visible to t
         if (report) flag_error(a.err, CSA_DEVERR_INDEX);
         return -1;
     }
@@ -440,20 +440,32 @@ bool encode_rows512(CUtensorMap *m, const void *base, uint64_t rows, uint32_t bo
 
 } // namespace
 
-cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled)
+cudaError_t launch_attn_prefill_pair(const PrefillArgs &a, cudaStream_t st, bool *handled);
+
+cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled, bool *pair)
 {
     *handled = false;
+    *pair = false;
+    if (!a.idx) { // HCA (every visible entry): two tokens per item on a 2-CTA cluster
+        cudaError_t e = launch_attn_prefill_pair(a, st, pair);
+        if (*pair) {
+            *handled = true;
+            return e;
+        }
+    }
     if (a.dtype != CSA_BF16 || a.H != kH || a.c != kC || a.W != kW || a.T <= 0) return cudaSuccess;
     if (a.idx && a.k > 4096) return cudaSuccess;
     if ((uint64_t)a.T * kH >= (1ull << 31)) return cudaSuccess; // TMA row coordinates are int32
+    // from here on the call is this kernel's: a tensor map that cannot be encoded is an error
+    // (reported as a failed launch), never a silent switch to the CUDA-core kernel
+    *handled = true;
     TmaMaps maps;
     if (!encode_rows512(&maps.q, a.q, (uint64_t)a.T * kH, 64) || !encode_rows512(&maps.x, a.x_win, (uint64_t)a.T, kKT))
-        return cudaSuccess; // no tensor-map encoder: the generic path serves the call
+        return cudaErrorNotSupported;
     const bool have_kv = a.kv_comp != nullptr && a.n_comp > 0;
     if (!encode_rows512(&maps.kv, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, kKT) ||
         !encode_rows512(&maps.kvg, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, 1))
-        return cudaSuccess;
-    *handled = true;
+        return cudaErrorNotSupported;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;

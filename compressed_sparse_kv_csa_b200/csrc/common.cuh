@@ -122,6 +122,17 @@ __device__ __forceinline__ int fp4_scale_exp(float amax)
     return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
+// Row of compressed entry s of sequence / query b in a paged cache (-1 when the page index is out
+// of the table), else the contiguous row base + s.
+__device__ __forceinline__ int64_t paged_row(const int32_t *pages, int max_pages, int page_rows, int64_t b, int64_t s,
+                                             int64_t base)
+{
+    if (!pages) return base + s;
+    const int64_t pg = s / page_rows;
+    if (pg >= max_pages) return -1;
+    return (int64_t)pages[b * max_pages + pg] * page_rows + s % page_rows;
+}
+
 // fp32 order-preserving key: larger float -> larger unsigned key.
 __device__ __forceinline__ uint32_t float_key(float f)
 {
@@ -154,6 +165,7 @@ __device__ __forceinline__ float warp_max(float v)
 namespace csa {
 
 int *dev_error_word(); // device address of the error word for the current device
+int device_sms();      // SM count of the current device
 
 struct KvRowsDev {
     uint8_t *fp8;
@@ -177,6 +189,15 @@ cudaError_t launch_quantize_kv(const void *x, int in_dtype, int64_t n, int c, in
                                const KvRowsDev &out, cudaStream_t st);
 cudaError_t launch_quantize_fp4(const void *x, int in_dtype, int64_t n, int d,
                                 const Fp4RowsDev &out, cudaStream_t st);
+cudaError_t launch_compress_append(bool overlap, int64_t B, const int64_t *pos, int c, int m, int in_dtype,
+                                   const void *const new_rows[4], void *const tail[4], const float *Bias,
+                                   const KvRowsDev *kv, const Fp4RowsDev *fp4, const int32_t *pages, int max_pages,
+                                   int page_rows, const int64_t *comp_off, int64_t n_out, int *err, cudaStream_t st);
+cudaError_t launch_window_append(const void *x, int in_dtype, int64_t B, int c, const int64_t *pos, int W,
+                                 const KvRowsDev &out, cudaStream_t st);
+cudaError_t launch_prep_rows(const void *x, int in_dtype, int64_t n, int d, const float *g, float eps, int rd,
+                             const int64_t *pos, double base, int hadamard, void *out, int out_dtype,
+                             const KvRowsDev *kv, const Fp4RowsDev *f4, cudaStream_t st);
 
 struct IndexerArgs {
     const void *q;        // dense [Nq,H,d] or null for fp4
@@ -189,12 +210,23 @@ struct IndexerArgs {
     int H, d, m, k;
     int64_t max_nvis, ld;  // ld: row stride of the score buffer
     float *scores;         // [Nq, ld] workspace
+    const int32_t *pages;  // paged keys: row of entry s of query r = pages[r*max_pages + s/page_rows]*page_rows + s%page_rows
+    int max_pages, page_rows;
     int32_t *idx_out;
     float *score_out;
     void *topk_ws;
     int *err;
 };
 cudaError_t launch_indexer_scores(const IndexerArgs &a, cudaStream_t st);
+
+// indexer_topk, indexer_topk_paged and indexer_topk_static: shared checks and launch (abi.cu).
+// scratch == nullptr: the caller's workspace must hold indexer_topk_workspace_size(); otherwise
+// ws_bytes is the static scratch's size and scratch() supplies its device address.
+int indexer_topk_impl(const void *q, const float *w, const void *keys, int32_t fmt, const int64_t *q_pos,
+                      const int64_t *key_off, int64_t n_keys, int64_t Nq, int32_t H_I, int32_t d_I, int32_t m,
+                      int32_t k, int64_t max_nvis, int32_t *idx_out, float *score_out, void *ws, size_t ws_bytes,
+                      void *(*scratch)(cudaError_t *), void *stream, const int32_t *pages = nullptr,
+                      int32_t max_pages = 0, int32_t page_rows = 0);
 cudaError_t launch_topk(const IndexerArgs &a, cudaStream_t st);
 
 struct PrefillArgs {
@@ -226,6 +258,9 @@ struct DecodeArgs {
     float *lse;
     float *part;          // split-K partials
     int n_chunks, chunk;  // chunks per sequence and keys per chunk
+    const int32_t *pages; // paged cache: row of entry s of sequence b = pages[b*max_pages + s/page_rows]*page_rows + s%page_rows
+    int max_pages, page_rows;
+    uint64_t wait_ns;     // limit of the tensor-core kernel's bounded waits
     int *err;
 };
 void decode_plan(int B, int H, int c, int max_keys, int *n_chunks, int *chunk);

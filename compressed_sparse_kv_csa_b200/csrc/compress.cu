@@ -30,6 +30,60 @@ struct CompressParams {
     bool has_fp4;
 };
 
+// Where the rows of an entry come from and where the entry goes.  Prefill: entry = the CTA slot,
+// token p is row p of the inputs, the entry is row `entry` of the outputs.
+struct PrefillRows {
+    int64_t n_entries;
+    __device__ bool entry(int64_t slot, int64_t &e) const
+    {
+        e = slot;
+        return slot < n_entries;
+    }
+    __device__ int64_t in_row(int64_t, int64_t p) const { return p; }
+    __device__ int64_t out_row(int64_t, int64_t e) const { return e; }
+};
+
+// Decode append: slot = sequence b, whose new token sits at position pos[b]; an entry is emitted
+// only when that token completes a block ((pos + 1) % m == 0, entry (pos + 1) / m - 1).  Token p
+// of sequence b is row b * L + p % L of the tail ring (the last L tokens' compressor rows); the
+// entry lands in the sequence's page (pages[b * max_pages + e / page_rows] * page_rows +
+// e % page_rows) or at comp_off[b] + e.  An entry whose page slot is missing or beyond the output
+// rows is skipped and reported (CSA_DEVERR_INDEX).
+struct AppendRows {
+    const int64_t *pos;
+    int64_t B;
+    int m, L;
+    const int32_t *pages;
+    int max_pages, page_rows;
+    const int64_t *comp_off;
+    int64_t n_out;
+    int *err;
+    __device__ bool entry(int64_t b, int64_t &e) const
+    {
+        if (b >= B) return false;
+        const int64_t t = pos[b];
+        if (t < 0 || (t + 1) % m != 0) return false;
+        e = (t + 1) / m - 1;
+        return true;
+    }
+    __device__ int64_t in_row(int64_t b, int64_t p) const { return b * L + p % L; }
+    __device__ int64_t out_row(int64_t b, int64_t e) const
+    {
+        int64_t r;
+        if (pages) {
+            const int64_t pg = e / page_rows;
+            r = pg < max_pages ? (int64_t)pages[b * max_pages + pg] * page_rows + e % page_rows : -1;
+        } else {
+            r = comp_off[b] + e;
+        }
+        if (r < 0 || r >= n_out) {
+            flag_error(err, CSA_DEVERR_INDEX);
+            return -1;
+        }
+        return r;
+    }
+};
+
 struct SoftState {
     float mx[4], den[4], num[4];
 };
@@ -63,14 +117,15 @@ __device__ __forceinline__ void soft_merge(SoftState &s, const float *o)
     }
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
+template <typename Tin, typename Rows>
+__global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS, Rows R)
 {
     extern __shared__ float smem[];
     const int TPE = blockDim.x; // channel groups of 4
     const int x = threadIdx.x, y = threadIdx.y, z = threadIdx.z;
-    const int64_t entry = (int64_t)blockIdx.x * blockDim.z + z;
-    const bool valid = entry < p.n_entries;
+    const int64_t slot = (int64_t)blockIdx.x * blockDim.z + z;
+    int64_t entry = 0;
+    bool valid = R.entry(slot, entry);
     const int ch = 4 * x;
     const int c = p.c, m = p.m;
 
@@ -85,7 +140,7 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
         const Tin *Ca = (const Tin *)p.Ca, *Za = (const Tin *)p.Za;
         const int j0 = (int)((int64_t)m * y / TS), j1 = (int)((int64_t)m * (y + 1) / TS);
         for (int j = j0; j < j1; ++j) { // current block
-            const int64_t row = entry * m + j;
+            const int64_t row = R.in_row(slot, entry * m + j);
             float4 v = Ld4<Tin>::at(Ca, row * c + ch);
             float4 zz = Ld4<Tin>::at(Za, row * c + ch);
             float4 b = *reinterpret_cast<const float4 *>(p.B + (int64_t)j * c + ch);
@@ -95,7 +150,7 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
         if (p.overlap && entry > 0) { // previous block (Cb / Zb, bias rows m..2m-1)
             const Tin *Cb = (const Tin *)p.Cb, *Zb = (const Tin *)p.Zb;
             for (int j = j0; j < j1; ++j) {
-                const int64_t row = (entry - 1) * m + j;
+                const int64_t row = R.in_row(slot, (entry - 1) * m + j);
                 float4 v = Ld4<Tin>::at(Cb, row * c + ch);
                 float4 zz = Ld4<Tin>::at(Zb, row * c + ch);
                 float4 b = *reinterpret_cast<const float4 *>(p.B + (int64_t)(m + j) * c + ch);
@@ -104,6 +159,9 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
             }
         }
     }
+    // output row of the entry (the policy may refuse it: nothing is written then)
+    int64_t orow = 0;
+    if (valid && y == 0 && x == 0) orow = R.out_row(slot, entry);
     // merge the token splits
     float *part = smem;                                       // [EPC][TS][TPE][12]
     int *amax_s = reinterpret_cast<int *>(smem + (size_t)blockDim.z * TS * TPE * 12); // [EPC]
@@ -116,16 +174,22 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
             mine[8 + u] = s.num[u];
         }
     }
-    if (x == 0 && y == 0) amax_s[z] = 0;
+    int64_t *orow_s = reinterpret_cast<int64_t *>(amax_s + 2 * blockDim.z); // [EPC], 8-byte aligned
+    if (x == 0 && y == 0) {
+        amax_s[z] = 0;
+        orow_s[z] = orow;
+    }
     __syncthreads();
+    orow = orow_s[z];
+    if (orow < 0) valid = false;
     float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
     if (y == 0) {
         for (int yy = 1; yy < TS; ++yy) soft_merge(s, part + (((size_t)z * TS + yy) * TPE + x) * 12);
         val = make_float4(s.num[0] / s.den[0], s.num[1] / s.den[1], s.num[2] / s.den[2],
                           s.num[3] / s.den[3]);
         if (valid && p.out) {
-            if (p.out_dtype == CSA_F32) st4<float>((float *)p.out, entry * c + ch, val);
-            else st4<uint16_t>((uint16_t *)p.out, entry * c + ch, val);
+            if (p.out_dtype == CSA_F32) st4<float>((float *)p.out, orow * c + ch, val);
+            else st4<uint16_t>((uint16_t *)p.out, orow * c + ch, val);
         }
         if (valid && p.has_kv && ch < c - p.kv.rope_dims) {
             float a = fmaxf(fmaxf(fabsf(val.x), fabsf(val.y)), fmaxf(fabsf(val.z), fabsf(val.w)));
@@ -146,11 +210,11 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
                          (uint32_t(e4m3_encode(__fdiv_rn(val.y, sc))) << 8) |
                          (uint32_t(e4m3_encode(__fdiv_rn(val.z, sc))) << 16) |
                          (uint32_t(e4m3_encode(__fdiv_rn(val.w, sc))) << 24);
-            *reinterpret_cast<uint32_t *>(p.kv.fp8 + entry * cn + ch) = w;
-            if (x == 0) p.kv.scale[entry] = sc;
+            *reinterpret_cast<uint32_t *>(p.kv.fp8 + orow * cn + ch) = w;
+            if (x == 0) p.kv.scale[orow] = sc;
         } else {
             const int rd = p.kv.rope_dims;
-            st4<uint16_t>(p.kv.rope, entry * rd + (ch - cn), val);
+            st4<uint16_t>(p.kv.rope, orow * rd + (ch - cn), val);
         }
     }
     if (p.has_fp4) {
@@ -164,10 +228,32 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams p, int TS)
         uint16_t two = uint16_t(e2m1x2_encode(val.x * inv, val.y * inv)) |
                        (uint16_t(e2m1x2_encode(val.z * inv, val.w * inv)) << 8);
         if (valid) {
-            *reinterpret_cast<uint16_t *>(p.fp4.codes + entry * (c / 2) + ch / 2) = two;
-            if ((x & 7) == 0) p.fp4.scales[entry * (c / 32) + ch / 32] = uint8_t(e + 127);
+            *reinterpret_cast<uint16_t *>(p.fp4.codes + orow * (c / 2) + ch / 2) = two;
+            if ((x & 7) == 0) p.fp4.scales[orow * (c / 32) + ch / 32] = uint8_t(e + 127);
         }
     }
+}
+
+// Block shape of the compression kernel: TPE = c / 4 threads per entry along the channels, TS
+// token splits for long HCA blocks, EPC entries per CTA.  The append path uses the same shape for
+// the same (overlap, c, m), so its entries are computed in the same order, bit for bit.
+static void compress_shape(bool overlap, int c, int m, int64_t n_entries, int *TS_, int *EPC_)
+{
+    const int TPE = c / 4;
+    int TS = 1;
+    if (!overlap && TPE >= 32) { // long HCA blocks: split the tokens of a block over threads
+        while (TS * 2 * TPE <= 512 && TS * 2 <= m && m / (TS * 2) >= 8) TS *= 2;
+    }
+    // whole warps only (the FP4 path shuffles with a full mask); extra entries are invalid lanes
+    int EPC = (TPE * TS >= 32) ? 1 : 32 / (TPE * TS);
+    while (EPC * 2 * TPE * TS <= 256 && EPC * 2 <= n_entries) EPC *= 2;
+    *TS_ = TS;
+    *EPC_ = EPC;
+}
+
+static size_t compress_smem(int EPC, int TS, int TPE)
+{
+    return (size_t)EPC * TS * TPE * 12 * sizeof(float) + (size_t)EPC * 2 * sizeof(int) + (size_t)EPC * sizeof(int64_t);
 }
 
 cudaError_t launch_compress(bool overlap, const void *Ca, const void *Cb, const void *Za,
@@ -185,20 +271,124 @@ cudaError_t launch_compress(bool overlap, const void *Ca, const void *Cb, const 
     if (fp4) p.fp4 = *fp4;
     if (p.n_entries == 0) return cudaSuccess;
     const int TPE = c / 4;
-    int TS = 1;
-    if (!overlap && TPE >= 32) { // long HCA blocks: split the tokens of a block over threads
-        while (TS * 2 * TPE <= 512 && TS * 2 <= m && m / (TS * 2) >= 8) TS *= 2;
-    }
-    // whole warps only (the FP4 path shuffles with a full mask); extra entries are invalid lanes
-    int EPC = (TPE * TS >= 32) ? 1 : 32 / (TPE * TS);
-    while (EPC * 2 * TPE * TS <= 256 && EPC * 2 <= p.n_entries) EPC *= 2;
+    int TS, EPC;
+    compress_shape(overlap, c, m, p.n_entries, &TS, &EPC);
     dim3 block(TPE, TS, EPC);
     const int64_t grid = (p.n_entries + EPC - 1) / EPC;
-    size_t smem = (size_t)EPC * TS * TPE * 12 * sizeof(float) + EPC * sizeof(int);
+    const size_t smem = compress_smem(EPC, TS, TPE);
+    const PrefillRows R{p.n_entries};
     if (in_dtype == CSA_F32)
-        compress_kernel<float><<<(unsigned)grid, block, smem, st>>>(p, TS);
+        compress_kernel<float, PrefillRows><<<(unsigned)grid, block, smem, st>>>(p, TS, R);
     else
-        compress_kernel<uint16_t><<<(unsigned)grid, block, smem, st>>>(p, TS);
+        compress_kernel<uint16_t, PrefillRows><<<(unsigned)grid, block, smem, st>>>(p, TS, R);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// decode append: tail ring of the compressor inputs, block completion, window ring
+// ------------------------------------------------------------------------------------------
+
+// Copy the new token's compressor rows (narr arrays of [B, c]) into slot pos[b] % L of sequence b's
+// tail ring ([B, L, c] per array).  8-byte moves (c a multiple of 4; bf16 rows are 8-byte aligned).
+template <typename T>
+__global__ void tail_one_kernel(const T *src, T *dst, const int64_t *pos, int c, int L)
+{
+    const int64_t b = blockIdx.x;
+    const int64_t t = pos[b];
+    if (t < 0) return;
+    const T *s = src + b * c;
+    T *d = dst + (b * L + t % L) * c;
+    constexpr int V = 8 / sizeof(T);
+    for (int i = threadIdx.x * V; i < c; i += blockDim.x * V)
+        *reinterpret_cast<uint2 *>(d + i) = *reinterpret_cast<const uint2 *>(s + i);
+}
+
+cudaError_t launch_compress_append(bool overlap, int64_t B, const int64_t *pos, int c, int m, int in_dtype,
+                                   const void *const new_rows[4], void *const tail[4], const float *Bias,
+                                   const KvRowsDev *kv, const Fp4RowsDev *fp4, const int32_t *pages, int max_pages,
+                                   int page_rows, const int64_t *comp_off, int64_t n_out, int *err, cudaStream_t st)
+{
+    if (B == 0) return cudaSuccess;
+    const int narr = overlap ? 4 : 2;
+    const int L = overlap ? 2 * m : m;
+    // 1. the new tokens into the tail rings, one launch per array
+    for (int a = 0; a < narr; ++a) {
+        if (in_dtype == CSA_F32)
+            tail_one_kernel<float><<<(unsigned)B, 128, 0, st>>>((const float *)new_rows[a], (float *)tail[a], pos, c, L);
+        else
+            tail_one_kernel<uint16_t><<<(unsigned)B, 128, 0, st>>>((const uint16_t *)new_rows[a], (uint16_t *)tail[a], pos, c,
+                                                                   L);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // 2. the entries completed by the new tokens, computed exactly as the prefill compression does
+    CompressParams p;
+    p.Ca = tail[0];
+    p.Cb = overlap ? tail[1] : nullptr;
+    p.Za = overlap ? tail[2] : tail[1];
+    p.Zb = overlap ? tail[3] : nullptr;
+    p.B = Bias;
+    p.T = 0;
+    p.n_entries = B;
+    p.c = c;
+    p.m = m;
+    p.overlap = overlap;
+    p.out = nullptr;
+    p.out_dtype = 0;
+    p.has_kv = kv != nullptr;
+    if (kv) p.kv = *kv;
+    p.has_fp4 = fp4 != nullptr;
+    if (fp4) p.fp4 = *fp4;
+    const int TPE = c / 4;
+    int TS, EPC;
+    compress_shape(overlap, c, m, B, &TS, &EPC);
+    dim3 block(TPE, TS, EPC);
+    const int64_t grid = (B + EPC - 1) / EPC;
+    const size_t smem = compress_smem(EPC, TS, TPE);
+    const AppendRows R{pos, B, m, L, pages, max_pages, page_rows, comp_off, n_out, err};
+    if (in_dtype == CSA_F32)
+        compress_kernel<float, AppendRows><<<(unsigned)grid, block, smem, st>>>(p, TS, R);
+    else
+        compress_kernel<uint16_t, AppendRows><<<(unsigned)grid, block, smem, st>>>(p, TS, R);
+    return cudaGetLastError();
+}
+
+// The new tokens' raw KV rows into the window rings: row x[b] -> window row b * W + pos[b] % W,
+// quantised exactly as csa_quantize_kv quantises a row.  One warp per row.
+template <typename Tin>
+__global__ void window_append_kernel(const Tin *x, int64_t B, int c, const int64_t *pos, int W, KvRowsDev out)
+{
+    const int64_t b = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (b >= B || pos[b] < 0) return;
+    const int64_t row = b * W + pos[b] % W;
+    const int rope = out.rope_dims, cn = c - rope;
+    float a = 0.f;
+    for (int j = lane * 4; j < cn; j += 128) {
+        float4 v = Ld4<Tin>::at(x, b * c + j);
+        a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    a = warp_max(a);
+    float sc = __fdiv_rn(a, 448.f);
+    if (!(sc > 0.f)) sc = 1.f;
+    for (int j = lane * 4; j < cn; j += 128) {
+        float4 v = Ld4<Tin>::at(x, b * c + j);
+        uint32_t w = uint32_t(e4m3_encode(__fdiv_rn(v.x, sc))) | (uint32_t(e4m3_encode(__fdiv_rn(v.y, sc))) << 8) |
+                     (uint32_t(e4m3_encode(__fdiv_rn(v.z, sc))) << 16) |
+                     (uint32_t(e4m3_encode(__fdiv_rn(v.w, sc))) << 24);
+        *reinterpret_cast<uint32_t *>(out.fp8 + row * cn + j) = w;
+    }
+    for (int j = lane * 4; j < rope; j += 128) st4<uint16_t>(out.rope, row * rope + j, Ld4<Tin>::at(x, b * c + cn + j));
+    if (lane == 0) out.scale[row] = sc;
+}
+
+cudaError_t launch_window_append(const void *x, int in_dtype, int64_t B, int c, const int64_t *pos, int W,
+                                 const KvRowsDev &out, cudaStream_t st)
+{
+    if (B == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((B + 7) / 8);
+    if (in_dtype == CSA_F32) window_append_kernel<float><<<grid, 256, 0, st>>>((const float *)x, B, c, pos, W, out);
+    else window_append_kernel<uint16_t><<<grid, 256, 0, st>>>((const uint16_t *)x, B, c, pos, W, out);
     return cudaGetLastError();
 }
 

@@ -19,13 +19,19 @@
 //   * MMA lane: copies the tile's scale words into TMEM (tcgen05.cp 32x128b.warpx4), then two
 //     M=128 (keys) x N=64 (heads) x K=64 block-scaled MMAs into one of four TMEM accumulators;
 //   * 8 epilogue warps in two groups taking alternate tiles (one key per lane, a warp per TMEM
-//     lane quadrant): score = w . ReLU(row of 64 head dot products), then a
-//     streaming filter: a key enters the chunk's candidate buffer only if it beats the current
-//     k-th best; every 4 tiles, if the buffer is nearly full, an exact radix selection cuts it
-//     back to k and raises the bar.  At the end the chunk's exact top-min(k, n) leave as 64-bit candidates
-//     (score key << 32 | ~entry, so equal scores order the lower entry first).
-// Kernel 2 (one CTA per query): the exact top-k of the union of its chunks' candidates (the
-//   global top-k is contained in it), sorted by score descending then entry ascending.
+//     lane quadrant): score = w . ReLU(row of 64 head dot products), written to the score
+//     buffer, and kept in the thread's own top-R list (registers, 64-bit keys
+//     score key << 32 | ~entry, so equal scores order the lower entry first) when it beats the
+//     list's last key.  No barrier inside the tile loop.
+//   At the end of the chunk the lists (256 x R keys) are cut to about p = the chunk's share of k
+//   (one radix digit, or an exact selection when that digit keeps too many) and published with
+//   the chunk's bound theta_c: every key of the chunk that is not published is below theta_c
+//   (theta_c = 0 when every key is published).
+// Kernel 2 (one CTA per query): theta = the k-th largest published key is at most the query's
+//   true k-th largest key (the k-th of a subset), so the exact top-k lies among the keys >= theta.
+//   A chunk with theta_c <= theta published all of those; the others ("saturated", rare: a chunk
+//   holding far more than its share of the winners) are re-read whole from the score buffer.  The
+//   exact top-k of that set is then sorted by score descending, entry ascending.
 // Every wait is bounded (%globaltimer); a timeout sets CSA_DEVERR_TIMEOUT and the CTA winds down.
 #include "common.cuh"
 #include "select.cuh"
@@ -42,8 +48,8 @@ using namespace tc;
 
 constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 8;
 constexpr int kChunk = 16384;                 // most keys per CTA
-constexpr int kCap = 4096;                    // candidate buffer (> k + kCheck tiles for k <= 2048)
-constexpr int kCheck = 4;                     // tiles between checks of the buffer's fill
+constexpr int kR = 8;                         // keys kept per epilogue thread
+constexpr int kMergeSmem = 200 * 1024;        // merge kernel: published lists + winners
 constexpr int kProdWarp = 0, kEpiWarp0 = 1, kEpiWarps = 8, kMmaWarp = kEpiWarp0 + kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -54,8 +60,8 @@ constexpr uint32_t OFF_ST = 0;                              // 8 x 8 KB codes (6
 constexpr uint32_t OFF_Q = OFF_ST + kStages * kTileCodes;    // query codes [64 x 64 B]
 constexpr uint32_t OFF_SCL = OFF_Q + 4096;                   // 8 x 128 scale words, then the query's
 constexpr uint32_t OFF_W = OFF_SCL + (kStages + 1) * 512;    // w [64] fp32
-constexpr uint32_t OFF_BUF = OFF_W + 256;                    // 2 x kCap candidates
-constexpr uint32_t OFF_SEL = OFF_BUF + 2 * kCap * 8;         // selection scratch (< 2 KB)
+constexpr uint32_t OFF_BUF = OFF_W + 256;                    // the threads' lists, 256 x kR keys
+constexpr uint32_t OFF_SEL = OFF_BUF + kEpiThreads * kR * 8; // selection scratch (< 2 KB)
 constexpr uint32_t OFF_MISC = OFF_SEL + 2048;                // counters
 constexpr uint32_t OFF_BAR = OFF_MISC + 256;
 constexpr uint32_t OFF_TMEM = OFF_BAR + 512;
@@ -74,10 +80,10 @@ enum { B_FULL = 0, B_EMPTY = B_FULL + kStages, B_DFULL = B_EMPTY + kStages, B_DE
 static_assert(NUM_BARS * 8 <= 512, "barrier space");
 static_assert(sizeof(SelectSmem<uint32_t>) <= 2048, "selection scratch");
 
-enum { M_COUNT = 0, M_ABORT = 1, M_OUT = 2 };
+enum { M_COUNT = 0, M_ABORT = 1, M_OUT = 2, M_RED = 4 }; // M_RED: 8 x u64 (one per warp)
 
 struct Maps {
-    CUtensorMap q, k;
+    CUtensorMap q, k, kp; // kp: key rows in boxes of one page (paged caches only)
 };
 
 __device__ __forceinline__ int64_t dec_nvis(const IndexerArgs &a, int64_t r)
@@ -85,6 +91,10 @@ __device__ __forceinline__ int64_t dec_nvis(const IndexerArgs &a, int64_t r)
     const int64_t t = a.q_pos ? a.q_pos[r] : r;
     int64_t nv = (t + 1) / a.m;
     if (nv > a.max_nvis) nv = a.max_nvis;
+    if (a.pages) { // the page table bounds the entries
+        const int64_t cap = (int64_t)a.max_pages * a.page_rows;
+        return nv < 0 ? 0 : (nv > cap ? cap : nv);
+    }
     const int64_t base = a.key_off ? a.key_off[r] : 0;
     if (base < 0) return 0;
     if (nv > a.n_keys - base) nv = a.n_keys - base;
@@ -100,11 +110,43 @@ __device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity)
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kEpiBar), "n"(kEpiThreads) : "memory"); }
 
 // ------------------------------------------------------------------------------------------
-// kernel 1: FP4 key scan (tcgen05 kind::mxf4) + streaming chunk top-k
+// kernel 1: FP4 key scan (tcgen05 kind::mxf4), every score stored, per-thread top-R lists
 // ------------------------------------------------------------------------------------------
+
+// Chunk output: list [lcap] 64-bit keys, count, theta_c (every unpublished key of the chunk is
+// below theta_c; 0 when all are published).
+struct ChunkOut {
+    unsigned long long *list;   // [Nq, n_slots, lcap]
+    int *count;                 // [Nq, n_slots]
+    unsigned long long *theta;  // [Nq, n_slots]
+    int n_slots, chunk, lcap, keep;
+};
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
+// Largest of one value per epilogue thread (all 256 call it; returns the same on all).
+__device__ __forceinline__ unsigned long long epi_max_u64(unsigned long long v, unsigned long long *red, int etid)
+{
+    v = warp_max_u64(v);
+    if ((etid & 31) == 0) red[etid >> 5] = v;
+    epi_sync();
+    unsigned long long m = red[0];
+#pragma unroll
+    for (int w = 1; w < kEpiWarps; ++w) m = red[w] > m ? red[w] : m;
+    epi_sync(); // red is read by every thread before it is reused
+    return m;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a, const __grid_constant__ Maps maps,
-                                                                  int n_slots, int chunk, unsigned long long *cand,
-                                                                  int *cand_count)
+                                                                  ChunkOut co)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -114,18 +156,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t r = blockIdx.y;
     const int slot = blockIdx.x;
+    const int chunk = co.chunk;
     const int64_t nv = dec_nvis(a, r);
     const int64_t c0 = (int64_t)slot * chunk;
     const int n = (int)(nv - c0 < chunk ? (nv - c0 > 0 ? nv - c0 : 0) : chunk);
-    unsigned long long *out = cand + ((int64_t)r * n_slots + slot) * a.k;
-    int *out_count = cand_count + r * n_slots + slot;
+    const int64_t oslot = r * co.n_slots + slot;
+    unsigned long long *out = co.list + oslot * co.lcap;
     if (n == 0) { // nothing visible in this chunk (CTA-uniform)
-        if (tid == 0) *out_count = 0;
+        if (tid == 0) {
+            co.count[oslot] = 0;
+            co.theta[oslot] = 0ull;
+        }
         return;
     }
     const int64_t key0 = (a.key_off ? a.key_off[r] : 0) + c0; // first key row of the chunk
     const int ntiles = (n + kKT - 1) / kKT;
     int *misc = reinterpret_cast<int *>(sp + OFF_MISC);
+    unsigned long long *red = reinterpret_cast<unsigned long long *>(sp + OFF_MISC + 4 * M_RED);
 
     if (tid == 0) {
         for (int b = 0; b < NUM_BARS; ++b) {
@@ -164,101 +211,138 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             if (i >= kStages && !wwait(bar(B_EMPTY + st), ((i / kStages) - 1) & 1)) { ok = false; break; }
             const int64_t row0 = key0 + (int64_t)i * kKT;
             const int valid = n - i * kKT < kKT ? n - i * kKT : kKT; // keys of the chunk in this tile
-            for (int j = lane; j < valid; j += 32)
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + OFF_SCL + st * 512u +
-                                                                          16u * (j & 31) + 4u * (j >> 5)),
-                             "l"(scales + row0 + j)
-                             : "memory");
+            const int64_t e0 = c0 + (int64_t)i * kKT;                // the tile's first entry
+            for (int j = lane; j < valid; j += 32) {
+                const int64_t row = a.pages ? paged_row(a.pages, a.max_pages, a.page_rows, r, e0 + j, 0) : row0 + j;
+                if (row >= 0 && row < a.k4.n) // a bad page leaves the word unset; the epilogue drops the key
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + OFF_SCL + st * 512u +
+                                                                              16u * (j & 31) + 4u * (j >> 5)),
+                                 "l"(scales + row)
+                                 : "memory");
+            }
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_FULL + st)) : "memory");
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(B_FULL + st), kTileCodes);
-                tma_load_2d(base + OFF_ST + st * kTileCodes, &maps.k, 0, (int32_t)row0, bar(B_FULL + st));
+                if (!a.pages) {
+                    tma_load_2d(base + OFF_ST + st * kTileCodes, &maps.k, 0, (int32_t)row0, bar(B_FULL + st));
+                } else { // one box per page; rows past the chunk or of a bad page read anything in range
+                    for (int u = 0; u * a.page_rows < kKT; ++u) {
+                        const int64_t eu = e0 + (int64_t)u * a.page_rows;
+                        int64_t row = eu < c0 + n ? paged_row(a.pages, a.max_pages, a.page_rows, r, eu, 0) : 0;
+                        if (row < 0 || row >= a.k4.n) row = 0;
+                        tma_load_2d(base + OFF_ST + st * kTileCodes + (uint32_t)(u * a.page_rows) * 64u, &maps.kp, 0,
+                                    (int32_t)row, bar(B_FULL + st));
+                    }
+                }
             }
         }
+        // every cp.async of this warp has landed before the CTA can exit
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp >= kEpiWarp0 && warp < kMmaWarp) {
         const int quad = warp & 3, etid = tid - 32 * kEpiWarp0, grp = (warp - kEpiWarp0) >> 2;
         float w[kHI];
 #pragma unroll
         for (int h = 0; h < kHI; ++h) w[h] = reinterpret_cast<const float *>(sp + OFF_W)[h];
-        unsigned long long *buf = reinterpret_cast<unsigned long long *>(sp + OFF_BUF);
-        unsigned long long *alt = buf + kCap;
-        SelectSmem<uint32_t> *sel = reinterpret_cast<SelectSmem<uint32_t> *>(sp + OFF_SEL);
-        unsigned long long theta = 0; // a key enters the buffer only above this
-        const int npairs = (ntiles + 1) / 2;
-        for (int p = 0; p < npairs; ++p) { // group g takes tile 2p + g; both groups pass the same barriers
-            const int i = 2 * p + grp;
+        float *srow = a.scores + r * a.ld + c0; // this chunk's scores
+        unsigned long long top[kR];             // this thread's best keys, descending (0 = empty)
+#pragma unroll
+        for (int j = 0; j < kR; ++j) top[j] = 0ull;
+        for (int i = grp; i < ntiles; i += 2) { // group g takes tiles g, g + 2, ...
             const uint32_t db = i % kDBufs;
-            const bool got = i >= ntiles || wwait(bar(B_DFULL + db), (i / kDBufs) & 1);
-            if (i >= ntiles) {
-            } else if (got) {
-                tc_fence_after();
-                uint32_t r0[32], r1[32];
-                const uint32_t ta = tmem + db * 64u + ((uint32_t)(32 * quad) << 16);
-                tmem_ld32(ta, r0);
-                tmem_ld32(ta + 32, r1);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
-                float acc[4] = {0.f, 0.f, 0.f, 0.f}; // four independent chains
+            if (!wwait(bar(B_DFULL + db), (i / kDBufs) & 1)) {
+                ok = false;
+                if (lane == 0) misc[M_ABORT] = 1;
+                break;
+            }
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            const uint32_t ta = tmem + db * 64u + ((uint32_t)(32 * quad) << 16);
+            tmem_ld32(ta, r0);
+            tmem_ld32(ta + 32, r1);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}; // four independent chains
 #pragma unroll
-                for (int h = 0; h < 32; ++h) acc[h & 3] = fmaf(w[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc[h & 3]);
+            for (int h = 0; h < 32; ++h) acc[h & 3] = fmaf(w[h], fmaxf(__uint_as_float(r0[h]), 0.f), acc[h & 3]);
 #pragma unroll
-                for (int h = 0; h < 32; ++h)
-                    acc[h & 3] = fmaf(w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc[h & 3]);
-                const float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                const int kc = i * kKT + 32 * quad + lane;
+            for (int h = 0; h < 32; ++h)
+                acc[h & 3] = fmaf(w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc[h & 3]);
+            const float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            const int kc = i * kKT + 32 * quad + lane;
+            bool live = kc < n;
+            if (live && a.pages) { // a key whose page is missing or out of range is dropped and reported
+                const int64_t row = paged_row(a.pages, a.max_pages, a.page_rows, r, c0 + kc, 0);
+                if (row < 0 || row >= a.k4.n) {
+                    flag_error(a.err, CSA_DEVERR_INDEX);
+                    srow[kc] = -INFINITY;
+                    live = false;
+                }
+            }
+            if (live) {
+                srow[kc] = s;
                 const unsigned long long cv =
                     ((unsigned long long)float_key(s) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)(c0 + kc));
-                const bool take = kc < n && cv > theta;
-                const unsigned bal = __ballot_sync(0xffffffffu, take);
-                if (bal) {
-                    int pos = 0;
-                    if (lane == 0) pos = atomicAdd(&misc[M_COUNT], __popc(bal));
-                    pos = __shfl_sync(0xffffffffu, pos, 0);
-                    if (take) buf[pos + __popc(bal & ((1u << lane) - 1u))] = cv;
+                if (cv > top[kR - 1]) { // insert, keeping the list sorted
+                    top[kR - 1] = cv;
+#pragma unroll
+                    for (int j = kR - 1; j > 0; --j) {
+                        const unsigned long long x = top[j - 1], y = top[j];
+                        top[j - 1] = y > x ? y : x;
+                        top[j] = y > x ? x : y;
+                    }
                 }
-            } else if (lane == 0) {
-                misc[M_ABORT] = 1;
-            }
-            if ((p + 1) % (kCheck / 2) != 0 && p + 1 != npairs) continue; // the buffer has room for kCheck tiles
-            epi_sync();
-            const bool abort = misc[M_ABORT] != 0;
-            const int cnt = misc[M_COUNT];
-            epi_sync(); // every warp has read the count before any appends the next tile's keys
-            if (abort) { ok = false; break; }
-            if (cnt > kCap - kCheck * kKT && cnt > a.k) { // cut the buffer back to the k best, raise the bar
-                theta = block_kth64<kEpiThreads, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
-                if (etid == 0) misc[M_OUT] = 0;
-                epi_sync();
-                for (int j = etid; j < cnt; j += kEpiThreads) {
-                    const unsigned long long v = buf[j];
-                    if (v >= theta) alt[atomicAdd(&misc[M_OUT], 1)] = v;
-                }
-                epi_sync();
-                for (int j = etid; j < a.k; j += kEpiThreads) buf[j] = alt[j];
-                if (etid == 0) misc[M_COUNT] = a.k;
-                epi_sync();
             }
         }
-        if (ok) { // the chunk's exact top-min(k, n)
-            const int cnt = misc[M_COUNT];
-            if (cnt > a.k) {
-                const unsigned long long thr =
-                    block_kth64<kEpiThreads, kEpiBar>(cnt, a.k, [&](int j) { return buf[j]; }, sel, etid);
-                if (etid == 0) misc[M_OUT] = 0;
-                epi_sync();
-                for (int j = etid; j < cnt; j += kEpiThreads) {
-                    const unsigned long long v = buf[j];
-                    if (v >= thr) out[atomicAdd(&misc[M_OUT], 1)] = v;
-                }
-                if (etid == 0) *out_count = a.k;
+        epi_sync();
+        if (misc[M_ABORT] != 0) ok = false; // uniform over the epilogue warps
+        if (ok) {
+            // 1. the lists into shared memory, densely; tau = the largest last key of a full list
+            unsigned long long *U = reinterpret_cast<unsigned long long *>(sp + OFF_BUF);
+            int mine = 0;
+#pragma unroll
+            for (int j = 0; j < kR; ++j) mine += top[j] != 0ull ? 1 : 0;
+            const int pos = atomicAdd(&misc[M_COUNT], mine);
+#pragma unroll
+            for (int j = 0; j < kR; ++j)
+                if (j < mine) U[pos + j] = top[j];
+            const unsigned long long tau = epi_max_u64(top[kR - 1], red, etid); // has a barrier: U complete
+            const int nu = misc[M_COUNT];
+            unsigned long long theta_c = tau;
+            int cnt;
+            if (nu <= co.keep) { // publish everything
+                for (int j = etid; j < nu; j += kEpiThreads) out[j] = U[j];
+                cnt = nu;
             } else {
-                for (int j = etid; j < cnt; j += kEpiThreads) out[j] = buf[j];
-                if (etid == 0) *out_count = cnt;
+                // 2. one radix digit of the high words keeps >= keep keys; an exact cut when it keeps too many
+                SelectSmem<uint32_t> *sel = reinterpret_cast<SelectSmem<uint32_t> *>(sp + OFF_SEL);
+                uint32_t kmin;
+                int lead, n_ge;
+                const int bin = top_bin32<kEpiThreads, kEpiBar>(
+                    nu, co.keep, [&](int j) { return (uint32_t)(U[j] >> 32); }, sel, kmin, lead, n_ge, etid);
+                unsigned long long thr = 0ull;
+                if (n_ge > co.lcap)
+                    thr = block_kth64<kEpiThreads, kEpiBar>(nu, co.keep, [&](int j) { return U[j]; }, sel, etid);
+                unsigned long long mx = 0ull; // the largest key that is not published
+                for (int j = etid; j < nu; j += kEpiThreads) {
+                    const unsigned long long v = U[j];
+                    const uint32_t hv = (uint32_t)(v >> 32) - kmin;
+                    const bool keep = thr ? v >= thr : (lead >= 32 ? 0 : (int)((hv << lead) >> 24)) >= bin;
+                    if (keep) out[atomicAdd(&misc[M_OUT], 1)] = v;
+                    else mx = v > mx ? v : mx;
+                }
+                mx = epi_max_u64(mx, red, etid); // has a barrier: M_OUT complete
+                cnt = misc[M_OUT];
+                if (mx != 0ull && mx + 1 > theta_c) theta_c = mx + 1;
+            }
+            if (etid == 0) {
+                co.count[oslot] = cnt;
+                co.theta[oslot] = theta_c;
             }
         } else if (etid == 0) {
-            *out_count = 0;
+            co.count[oslot] = 0;
+            co.theta[oslot] = ~0ull; // counts as saturated; the timeout flag marks the result invalid
         }
     } else if (warp == kMmaWarp && lane == 0) {
         ok = mbar_wait(bar(B_QFULL), 0);
@@ -295,110 +379,108 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
 }
 
 // ------------------------------------------------------------------------------------------
-// kernel 2: exact top-k over the chunk candidates of one query
+// kernel 2: exact top-k of one query from the published lists (and saturated chunks' scores)
 // ------------------------------------------------------------------------------------------
 constexpr int kMergeThreads = 1024;
+constexpr int kMaxSlots = 256;
 
-constexpr int kPivCap = 4096; // candidates above the sampled pivot that the merge selects from
-
-// pivot: the union is first filtered by a pivot taken from every 16th candidate (the 1.5 k / 16-th
-// best sample, which lies below the k-th best of the union with high probability), so the exact
-// selection runs on about 1.5 k candidates; when the filter keeps fewer than k or more than
-// kPivCap, the selection runs on the whole union.
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs a, int n_slots,
-                                                                     const unsigned long long *cand,
-                                                                     const int *cand_count, int pivot)
+__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a, ChunkOut co)
 {
     extern __shared__ unsigned long long mv[];
     __shared__ SelectSmem<uint32_t> msel;
-    __shared__ int s_cnt, s_off[64];
+    __shared__ int s_cnt, s_nsat, s_off[kMaxSlots + 1], s_sat_off[kMaxSlots + 1], s_sat_slot[kMaxSlots];
+    __shared__ unsigned long long s_theta[kMaxSlots];
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
-    const int k = a.k;
+    const int k = a.k, ns = co.n_slots, chunk = co.chunk;
+    const int64_t nv = dec_nvis(a, r);
     if (tid == 0) {
         int o = 0;
-        for (int s = 0; s < n_slots; ++s) {
-            s_off[s] = o;
-            o += cand_count[r * n_slots + s];
+        for (int sl = 0; sl < ns; ++sl) {
+            s_off[sl] = o;
+            o += co.count[r * ns + sl];
         }
-        s_cnt = o;
+        s_off[ns] = o;
+    }
+    for (int sl = tid; sl < ns; sl += kMergeThreads) s_theta[sl] = co.theta[r * ns + sl];
+    __syncthreads();
+    const int total = s_off[ns];
+    // 1. the published lists
+    for (int e = tid; e < ns * co.lcap; e += kMergeThreads) {
+        const int sl = e / co.lcap, i = e - sl * co.lcap;
+        if (i < s_off[sl + 1] - s_off[sl]) mv[s_off[sl] + i] = co.list[(r * ns + sl) * (int64_t)co.lcap + i];
     }
     __syncthreads();
-    const int total = s_cnt;
-    { // gather the chunk lists, 8 independent 8-byte loads per thread in flight
-        const unsigned long long *src = cand + r * n_slots * k;
-        const int span = n_slots * k;
-        for (int e0 = tid; e0 < span; e0 += 8 * kMergeThreads) {
-            unsigned long long v[8];
-            int dst[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * kMergeThreads;
-                dst[u] = -1;
-                if (e < span) {
-                    const int s = e / k, i = e - s * k;
-                    if (i < cand_count[r * n_slots + s]) {
-                        v[u] = src[e];
-                        dst[u] = s_off[s] + i;
-                    }
-                }
+    // 2. theta = the k-th largest published key (0 when fewer than k are published), then the
+    //    chunks that may hold unpublished keys >= theta
+    const unsigned long long theta =
+        total >= k ? block_kth64<kMergeThreads>(total, k, [&](int i) { return mv[i]; }, &msel) : 0ull;
+    if (tid == 0) {
+        int nsat = 0, o = 0;
+        for (int sl = 0; sl < ns; ++sl) {
+            if (s_theta[sl] > theta) {
+                const int64_t n_s = nv - (int64_t)sl * chunk < chunk ? nv - (int64_t)sl * chunk : chunk;
+                s_sat_slot[nsat] = sl;
+                s_sat_off[nsat] = o;
+                o += (int)(n_s > 0 ? n_s : 0);
+                ++nsat;
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (dst[u] >= 0) mv[dst[u]] = v[u];
         }
+        s_sat_off[nsat] = o;
+        s_nsat = nsat;
+        s_cnt = 0;
     }
     __syncthreads();
-    const int ke = total < k ? total : k;
-    unsigned long long *buf = mv + total;                   // candidates above the pivot
-    unsigned long long *sel = buf + (pivot ? kPivCap : 0);  // ke winners
-    if (total > k) {
-        bool done = false;
-        const int ns = total >> 4, ks = (3 * k) >> 5;
-        if (pivot && ks >= 1 && ns >= 2 * ks) {
-            const unsigned long long piv =
-                block_kth64<kMergeThreads>(ns, ks, [&](int i) { return mv[16 * i]; }, &msel);
-            if (tid == 0) s_cnt = 0;
-            __syncthreads();
-            for (int i = tid; i < total; i += kMergeThreads) {
-                const unsigned long long v = mv[i];
-                if (v >= piv) {
-                    const int p = atomicAdd(&s_cnt, 1);
-                    if (p < kPivCap) buf[p] = v;
-                }
-            }
-            __syncthreads();
-            const int c = s_cnt;
-            if (c >= k && c <= kPivCap) { // the k best of the union are all above the pivot
-                const unsigned long long thr =
-                    block_kth64<kMergeThreads>(c, k, [&](int i) { return buf[i]; }, &msel);
-                __syncthreads();
-                if (tid == 0) s_cnt = 0;
-                __syncthreads();
-                for (int i = tid; i < c; i += kMergeThreads) {
-                    const unsigned long long v = buf[i];
-                    if (v >= thr) sel[atomicAdd(&s_cnt, 1)] = v;
-                }
-                done = true;
-            }
-            __syncthreads();
+    const int nsat = s_nsat;
+    unsigned long long *sel = mv + total; // the winners, padded to a power of two
+    int ke;
+    if (nsat == 0) { // every key >= theta is published: exactly min(k, total) of them
+        ke = total < k ? total : k;
+        for (int i = tid; i < total; i += kMergeThreads) {
+            const unsigned long long v = mv[i];
+            if (v >= theta) sel[atomicAdd(&s_cnt, 1)] = v;
         }
-        if (!done) {
-            const unsigned long long thr = block_kth64<kMergeThreads>(total, k, [&](int i) { return mv[i]; }, &msel);
-            if (tid == 0) s_cnt = 0;
-            __syncthreads();
-            for (int i = tid; i < total; i += kMergeThreads) {
-                const unsigned long long v = mv[i];
-                if (v >= thr) {
-                    const int p = atomicAdd(&s_cnt, 1);
-                    if (p < ke) sel[p] = v;
-                }
-            }
-        }
+        __syncthreads();
     } else {
-        for (int i = tid; i < total; i += kMergeThreads) sel[i] = mv[i];
+        // 3. saturated chunks join whole, from the stored scores (their published keys are dropped)
+        for (int j = 0; j < nsat; ++j) {
+            const int sl = s_sat_slot[j];
+            for (int i = s_off[sl] + tid; i < s_off[sl + 1]; i += kMergeThreads) mv[i] = 0ull;
+        }
+        __syncthreads();
+        const int nvirt = total + s_sat_off[nsat];
+        const float *srow = a.scores + r * a.ld;
+        auto get = [&](int i) -> unsigned long long {
+            if (i < total) return mv[i];
+            i -= total;
+            int j = 0;
+            while (j + 1 < nsat && i >= s_sat_off[j + 1]) ++j;
+            const int64_t e = (int64_t)s_sat_slot[j] * chunk + (i - s_sat_off[j]);
+            return ((unsigned long long)float_key(srow[e]) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)e);
+        };
+        int live = 0; // keys in the set (the dropped ones read 0)
+        for (int i = tid; i < nvirt; i += kMergeThreads) live += get(i) != 0ull ? 1 : 0;
+        for (int o = 16; o > 0; o >>= 1) live += __shfl_xor_sync(0xffffffffu, live, o);
+        if ((tid & 31) == 0) atomicAdd(&s_cnt, live);
+        __syncthreads();
+        const int n_live = s_cnt;
+        __syncthreads();
+        ke = n_live < k ? n_live : k;
+        // the k-th largest of the set (zeros sort below every key, so they never reach it)
+        const unsigned long long thr =
+            n_live > k ? block_kth64<kMergeThreads>(nvirt, k, get, &msel) : 1ull;
+        if (tid == 0) s_cnt = 0;
+        __syncthreads();
+        for (int i = tid; i < nvirt; i += kMergeThreads) {
+            const unsigned long long v = get(i);
+            if (v != 0ull && v >= thr) {
+                const int p = atomicAdd(&s_cnt, 1);
+                if (p < ke) sel[p] = v;
+            }
+        }
+        __syncthreads();
     }
-    __syncthreads();
+    // 4. order the winners: score descending, then entry ascending (bitonic sort of the 64-bit keys)
     int n2 = 1;
     while (n2 < ke) n2 <<= 1;
     for (int i = ke + tid; i < n2; i += kMergeThreads) sel[i] = 0ull;
@@ -429,71 +511,104 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(IndexerArgs
     }
 }
 
-} // namespace
+// Chunking of the key lists: at most one CTA per SM (the CTAs of one launch fill a single wave),
+// at most kChunk keys each; each chunk publishes `keep` keys (about twice its share of k, at
+// least 64) in a list of lcap slots sized so the merge holds every list in shared memory.
+struct Plan {
+    int slots, chunk, keep, lcap;
+};
 
-// Chunking of the key lists: at most one CTA per SM of the B200's 148 (the CTAs of one launch fill
-// a single wave: a 149th CTA would double the launch time), at most kChunk keys each.
-static void decode_chunks(int64_t Nq, int64_t max_nvis, int *slots, int *chunk)
+bool scan_plan(int64_t Nq, int64_t max_nvis, int k, int sms, Plan *p)
 {
-    int64_t want = 148 / (Nq > 0 ? Nq : 1);
+    int64_t want = sms / (Nq > 0 ? Nq : 1);
     if (want < 1) want = 1;
     int64_t ch = (max_nvis + want - 1) / want;
     ch = (ch + kKT - 1) / kKT * kKT;
     if (ch > kChunk) ch = kChunk;
     if (ch < kKT) ch = kKT;
-    *chunk = (int)ch;
-    *slots = (int)((max_nvis + ch - 1) / ch);
-    if (*slots < 1) *slots = 1;
+    p->chunk = (int)ch;
+    p->slots = (int)((max_nvis + ch - 1) / ch);
+    if (p->slots < 1) p->slots = 1;
+    const int share = (k + p->slots - 1) / p->slots;
+    p->keep = 2 * share + 32 > 64 ? 2 * share + 32 : 64;
+    if (p->keep > k) p->keep = k;
+    int n2 = 1;
+    while (n2 < k) n2 <<= 1;
+    const int64_t room = (kMergeSmem - (int64_t)n2 * 8) / ((int64_t)p->slots * 8);
+    p->lcap = (int)(room < 512 ? room : 512);
+    return p->slots <= kMaxSlots && p->lcap >= p->keep;
 }
 
-// Workspace bytes of the decode path (candidates + counts).
+size_t lists_bytes(int64_t Nq, const Plan &p)
+{
+    return ((size_t)Nq * (size_t)p.slots * ((size_t)p.lcap * 8 + 8 + 4) + 255) / 256 * 256;
+}
+
+} // namespace
+
+// Scratch of the decode path for this device: the chunk lists, counts and bounds, then every
+// score ([Nq, ceil4(max_nvis)] fp32, re-read by the merge for saturated chunks).
+size_t decode_indexer_need(int64_t Nq, int64_t max_nvis, int k)
+{
+    Plan p;
+    scan_plan(Nq, max_nvis, k, device_sms(), &p);
+    const size_t ld = (size_t)((max_nvis + 3) / 4 * 4);
+    return lists_bytes(Nq, p) + (size_t)Nq * ld * 4 + 256;
+}
+
+// A bound of decode_indexer_need on any device: the merge keeps every list in kMergeSmem bytes,
+// so the lists of one query never exceed that.
 size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k)
 {
-    int slots, chunk;
-    decode_chunks(Nq, max_nvis, &slots, &chunk);
-    return (size_t)Nq * (size_t)slots * ((size_t)k * 8 + 4) + 256;
+    (void)k;
+    const size_t ld = (size_t)((max_nvis + 3) / 4 * 4);
+    return (size_t)Nq * ((size_t)kMergeSmem + (size_t)kMaxSlots * 12 + 256) + (size_t)Nq * ld * 4 + 512;
 }
 
 bool decode_indexer_eligible(const IndexerArgs &a)
 {
     if (a.fmt != CSA_FP4 || a.H != kHI || a.d != kDI || a.Nq <= 0 || a.Nq > 65535 || a.max_nvis <= 0) return false;
+    if (a.pages && (a.page_rows < 8 || a.page_rows > kKT || (a.page_rows & (a.page_rows - 1)))) return false;
     if (a.k > 2048 || a.k4.n >= (1ll << 31) || a.Nq * kHI >= (1ll << 31)) return false;
-    int slots, chunk;
-    decode_chunks(a.Nq, a.max_nvis, &slots, &chunk);
-    if (slots > 64) return false;
-    // merge kernel: candidates (slots * k) plus the padded winner array must fit in shared memory
-    int n2 = 1;
-    while (n2 < a.k) n2 <<= 1;
-    return (size_t)(slots * a.k + n2) * 8 <= 200 * 1024;
+    Plan p;
+    return scan_plan(a.Nq, a.max_nvis, a.k, device_sms(), &p);
 }
 
-cudaError_t launch_indexer_decode(const IndexerArgs &a, void *ws, cudaStream_t st)
+cudaError_t launch_indexer_decode(const IndexerArgs &a0, void *ws, cudaStream_t st)
 {
-    int slots, chunk;
-    decode_chunks(a.Nq, a.max_nvis, &slots, &chunk);
-    uintptr_t p = (reinterpret_cast<uintptr_t>(ws) + 255) / 256 * 256;
-    unsigned long long *cand = reinterpret_cast<unsigned long long *>(p);
-    int *cnt = reinterpret_cast<int *>(cand + (size_t)a.Nq * slots * a.k);
+    Plan p;
+    if (!scan_plan(a0.Nq, a0.max_nvis, a0.k, device_sms(), &p)) return cudaErrorInvalidValue;
+    uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + 255) / 256 * 256;
+    ChunkOut co;
+    co.list = reinterpret_cast<unsigned long long *>(base);
+    co.theta = co.list + (size_t)a0.Nq * p.slots * p.lcap;
+    co.count = reinterpret_cast<int *>(co.theta + (size_t)a0.Nq * p.slots);
+    co.n_slots = p.slots;
+    co.chunk = p.chunk;
+    co.lcap = p.lcap;
+    co.keep = p.keep;
+    IndexerArgs a = a0;
+    a.scores = reinterpret_cast<float *>(base + lists_bytes(a0.Nq, p));
+    a.ld = (a0.max_nvis + 3) / 4 * 4;
     Maps maps;
     memset(&maps, 0, sizeof(maps));
     const uint64_t key_rows = a.k4.n > 0 ? (uint64_t)a.k4.n : 1; // an empty key array is never read
     if (!tma::encode_u8_rows_sw64(&maps.q, a.q4.codes, (uint64_t)a.Nq * kHI, kDI / 2, kHI) ||
         !tma::encode_u8_rows_sw64(&maps.k, a.k4.codes, key_rows, kDI / 2, kKT))
         return cudaErrorInvalidValue;
+    if (a.pages && !tma::encode_u8_rows_sw64(&maps.kp, a.k4.codes, key_rows, kDI / 2, (uint32_t)a.page_rows))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    decode_scan_kernel<<<dim3((unsigned)slots, (unsigned)a.Nq), kThreads, SMEM_ALLOC, st>>>(a, maps, slots, chunk, cand,
-                                                                                           cnt);
+    decode_scan_kernel<<<dim3((unsigned)p.slots, (unsigned)a.Nq), kThreads, SMEM_ALLOC, st>>>(a, maps, co);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int n2 = 1;
     while (n2 < a.k) n2 <<= 1;
-    size_t msm = (size_t)(slots * a.k + n2) * 8;
-    const int pivot = msm + (size_t)kPivCap * 8 <= 220 * 1024 ? 1 : 0;
-    if (pivot) msm += (size_t)kPivCap * 8;
-    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msm);
+    const size_t msm = (size_t)p.slots * p.lcap * 8 + (size_t)n2 * 8;
+    e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msm);
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<(unsigned)a.Nq, kMergeThreads, msm, st>>>(a, slots, cand, cnt, pivot);
+    topk_merge_kernel<<<(unsigned)a.Nq, kMergeThreads, msm, st>>>(a, co);
     return cudaGetLastError();
 }
 

@@ -221,11 +221,11 @@ cudaError_t launch_indexer_scores_tc(const IndexerArgs &a, cudaStream_t st, bool
     if (a.fmt != CSA_BF16 || a.H != kHI || a.d != kDI || a.q_pos || a.key_off || a.Nq <= 0 || a.n_keys <= 0)
         return cudaSuccess;
     if ((uint64_t)a.Nq * kHI >= (1ull << 31) || a.n_keys >= (1ll << 31)) return cudaSuccess;
+    *handled = true; // the call is this kernel's: an encoding failure is an error, not a switch of kernels
     Maps maps;
     if (!tma::encode_bf16_rows(&maps.q, a.q, (uint64_t)a.Nq * kHI, kDI, 256) ||
         !tma::encode_bf16_rows(&maps.k, a.keys, (uint64_t)a.n_keys, kDI, kMK))
-        return cudaSuccess;
-    *handled = true;
+        return cudaErrorNotSupported;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;

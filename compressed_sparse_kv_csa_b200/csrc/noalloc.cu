@@ -13,9 +13,8 @@
 
 namespace {
 
-// 4 Mi fp32 scores (16 MiB) plus one alignment slot of the workspace carving.
-constexpr size_t kStaticScores = size_t(4) << 20;
-constexpr size_t kStaticBytes = kStaticScores * sizeof(float) + 256;
+// 16 MiB of scratch plus one alignment slot of the workspace carving.
+constexpr size_t kStaticBytes = (size_t(16) << 20) + 256;
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kStaticBytes];
 
@@ -46,25 +45,18 @@ void *scratch_for_current_device(cudaError_t *err)
 
 extern "C" {
 
-size_t indexer_topk_static_capacity(void) { return kStaticScores; }
+size_t indexer_topk_static_capacity(void) { return kStaticBytes; }
 
 int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t fmt,
                         const int64_t *q_pos, const int64_t *key_off, int64_t n_keys, int64_t Nq,
                         int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis,
                         int32_t *idx_out, float *score_out, void *stream)
 {
-    if (Nq < 0 || max_nvis < 0) return CSA_ERR_INVALID_ARG;
-    if (Nq == 0) // nothing to score: the arguments are still checked, no device is needed
-        return indexer_topk(q, w, keys, fmt, q_pos, key_off, n_keys, Nq, H_I, d_I, m, k, max_nvis,
-                            idx_out, score_out, nullptr, 0, stream);
-    const size_t need = indexer_topk_workspace_size(Nq, max_nvis, k);
-    if (need > kStaticBytes) return CSA_ERR_SCRATCH_CAPACITY;
-    cudaError_t err = cudaSuccess;
-    void *scratch = scratch_for_current_device(&err);
-    if (!scratch) return CSA_ERR_CUDA;
-    // The scores are written before they are read within one call, so nothing is cleared.
-    return indexer_topk(q, w, keys, fmt, q_pos, key_off, n_keys, Nq, H_I, d_I, m, k, max_nvis, idx_out,
-                        score_out, scratch, kStaticBytes, stream);
+    // The same checks and kernels as indexer_topk; the request is refused when the scratch of the
+    // path it takes does not fit in the static array.  Every score is written before it is read
+    // within one call, so nothing needs clearing between calls.
+    return csa::indexer_topk_impl(q, w, keys, fmt, q_pos, key_off, n_keys, Nq, H_I, d_I, m, k, max_nvis, idx_out,
+                                  score_out, nullptr, kStaticBytes, scratch_for_current_device, stream);
 }
 
 } // extern "C"

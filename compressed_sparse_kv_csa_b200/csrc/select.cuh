@@ -141,6 +141,70 @@ __device__ void block_kth(int n, int k, Get get, SelectSmem<K> *sm, K &thr, int 
     n_gt = k - rem;
 }
 
+// One radix digit of a selection, for a cut that may keep a few more keys than asked: the n
+// 32-bit keys get(i) (n >= 1) are offset by their minimum and left-aligned on the highest bit of
+// their range, and binned by the top 8 bits of the result.  Returns the highest bin b such that
+// at least `want` keys (1 <= want <= n) lie in bins >= b, with the bin rule in kmin / lead (a key
+// v lies in bin ((v - kmin) << lead) >> 24; lead = 32 puts every key in bin 0 when all are equal)
+// and the number of keys in bins >= b in n_ge.  Same calling rules as block_kth.
+template <int NT, int BAR = 0, typename Get>
+__device__ int top_bin32(int n, int want, Get get, SelectSmem<uint32_t> *sm, uint32_t &kmin, int &lead, int &n_ge,
+                         int ltid = threadIdx.x)
+{
+    const int lane = ltid & 31, wid = ltid >> 5;
+    uint32_t lo = 0xffffffffu, hi = 0;
+    for (int i = ltid; i < n; i += NT) {
+        const uint32_t v = get(i);
+        lo = v < lo ? v : lo;
+        hi = v > hi ? v : hi;
+    }
+    lo = warp_min_key(lo);
+    hi = warp_max_key(hi);
+    if (lane == 0) { sm->red[wid] = lo; sm->red[32 + wid] = hi; }
+    for (int i = ltid; i < 256; i += NT) sm->hist[i] = 0;
+    group_sync<NT, BAR>();
+    uint32_t a = sm->red[0], b = sm->red[32];
+    for (int w = 1; w < NT / 32; ++w) {
+        a = sm->red[w] < a ? sm->red[w] : a;
+        b = sm->red[32 + w] > b ? sm->red[32 + w] : b;
+    }
+    kmin = a;
+    lead = (b == a) ? 32 : __clz(b - a);
+    for (int i = ltid; i < n; i += NT) {
+        const uint32_t v = get(i) - kmin;
+        atomicAdd(&sm->hist[lead >= 32 ? 0 : (int)((v << lead) >> 24)], 1);
+    }
+    group_sync<NT, BAR>();
+    if (wid == 0) { // suffix scan from the top bin: lane l owns bins 255-8l .. 248-8l
+        int c[8], s = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { c[j] = sm->hist[255 - 8 * lane - j]; s += c[j]; }
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int excl = incl - s;
+        const bool cross = excl < want && incl >= want;
+        const unsigned who = __ballot_sync(0xffffffffu, cross);
+        if (cross && lane == __ffs(who) - 1) {
+            int cum = excl, j = 0;
+            for (; j < 7; ++j) {
+                if (cum + c[j] >= want) break;
+                cum += c[j];
+            }
+            sm->bin = 255 - 8 * lane - j;
+            sm->rem = cum + c[j];
+        }
+    }
+    group_sync<NT, BAR>();
+    const int bin = sm->bin;
+    n_ge = sm->rem;
+    group_sync<NT, BAR>(); // the scratch is read before anyone reuses it
+    return bin;
+}
+
 // The k-th largest of n unique 64-bit keys (1 <= k <= n): a 32-bit radix selection on the high
 // words, then -- only when several keys share the threshold's high word and not all of them are
 // needed -- a second one on the low words of those ties.  Same calling rules as block_kth.

@@ -59,10 +59,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking check of the phase of `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase of `parity` to complete, for at most `limit_ns`.  Returns false (and the
-// caller records CSA_DEVERR_TIMEOUT) when the limit runs out.
+// caller records CSA_DEVERR_TIMEOUT) when the limit runs out.  A limit of at most 1 ns makes the
+// wait one non-blocking test, which gives up unless the phase has already completed: the way a
+// test makes waits run out on purpose.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = 2000000000ull)
 {
+    if (limit_ns <= 1) return mbar_test_wait(bar, parity);
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {

@@ -149,6 +149,72 @@ int csa_quantize_kv(const void *x, int32_t in_dtype, int64_t n, int32_t c, int32
 int csa_quantize_fp4(const void *x, int32_t in_dtype, int64_t n, int32_t d,
                      const csa_fp4_rows *out, void *stream);
 
+/*
+ * Decode append path ([qa] Question 5, KV-cache management: the sliding window and the tail
+ * tokens of the block still being compressed form a fixed-size "state cache", and the compressed
+ * entries live in block-managed pages whose size is the least common multiple of the ratios --
+ * 128 tokens for m = 4 and m' = 128, i.e. 32 CSA entries or 1 HCA entry per page; [notes] Sec.
+ * 2.3 Compressor listing: the decode branch emits an entry when a block completes).  One call of
+ * each per layer and decode step, for a batch of B sequences whose new tokens sit at pos[b] (every
+ * earlier token of the sequence must have been appended, in order; pos[b] < 0 skips b).
+ *
+ * csa_window_append: x [B, c] (in_dtype) are the new tokens' raw KV rows; row b is quantised (as
+ * csa_quantize_kv does) into window row b * W + pos[b] % W of `win` (B * W rows): the ring of the
+ * last min(pos + 1, W) tokens that hybrid_attn_decode reads with win_len[b] = min(pos[b] + 1, W).
+ * Errors: CSA_ERR_INVALID_ARG for a null x or pos, B < 0, a bad dtype, x not 16-byte aligned, W
+ * outside [1, 1024] or a `win` that does not hold B * W rows of c; CSA_ERR_UNSUPPORTED for c not a
+ * multiple of 4 in [4, 4096].
+ *
+ * csa_compress_append: the new tokens' compressor rows -- overlap != 0 (CSA, as csa_compress):
+ * Ca, Cb, Za, Zb [B, c]; overlap == 0 (HCA, as hca_compress): Ca = C, Za = Z, Cb = Zb = NULL --
+ * go to slot pos[b] % L of sequence b's tail ring (tail_* [B, L, c] in in_dtype, L = 2m for CSA,
+ * m for HCA; the caller allocates them once and keeps them across steps; HCA uses tail_Ca and
+ * tail_Za only).  When pos[b] completes a block ((pos[b] + 1) % m == 0) the entry
+ * e = (pos[b] + 1) / m - 1 is pooled from the ring exactly as the prefill compression pools it
+ * (same arithmetic, same order: the entries are bit for bit those of csa_compress /
+ * hca_compress) and written, quantised, into exactly one of out_kv (FP8/BF16 rows) or out_fp4
+ * (FP4 rows, for index keys) at row
+ *     pages[b * max_pages + e / page_rows] * page_rows + e % page_rows   (pages != NULL)
+ *     comp_off[b] + e                                                       (pages == NULL)
+ * A row outside the output, or a page index >= max_pages, is skipped and sets CSA_DEVERR_INDEX.
+ * Bias is [2m, c] (CSA) or [m, c] (HCA) fp32, 16-byte aligned; row pointers 8-byte aligned.
+ * Errors: CSA_ERR_INVALID_ARG for a null pos or Bias, B < 0, a bad dtype, m outside [1, 64] (CSA)
+ * or [1, 1024] (HCA), a missing or misaligned row or tail pointer, not exactly one output, no
+ * pages and no comp_off, or an output struct whose shape does not match c; CSA_ERR_UNSUPPORTED for
+ * c not a multiple of 4 in [4, 2048].
+ */
+int csa_window_append(const void *x, int32_t in_dtype, int64_t B, int32_t c, const int64_t *pos, int32_t W,
+                      const csa_kv_rows *win, void *stream);
+int csa_compress_append(int32_t overlap, int64_t B, const int64_t *pos, int32_t c, int32_t m, int32_t in_dtype,
+                        const void *Ca, const void *Cb, const void *Za, const void *Zb, void *tail_Ca,
+                        void *tail_Cb, void *tail_Za, void *tail_Zb, const float *Bias, const csa_kv_rows *out_kv,
+                        const csa_fp4_rows *out_fp4, const int32_t *pages, int32_t max_pages, int32_t page_rows,
+                        const int64_t *comp_off, void *stream);
+
+/*
+ * csa_prep_rows -- the per-row transforms between a projection and the caches ([notes] Sec. 2.3:
+ * the Compressor listing's RMSNorm of its entries; the Indexer listing's rotary embedding of
+ * q[..., -rd:], rotate_activation (Hadamard) and FP4 quantisation, which the indexer's own
+ * compressor (rotate=True) applies to its keys as well).  For each row r of x [n, d]:
+ *   y = x[r]
+ *   y = y / sqrt(mean(y^2) + eps) * g                 when g != NULL (g [d] fp32)
+ *   y[d-rd+2i], y[d-rd+2i+1] rotated by the angle      when rd > 0: counter-clockwise by
+ *       a = pos[r] * base^(-2i/rd)                     (pos [n] int64 positions)
+ *   y = y H_d / sqrt(d)                                when hadamard != 0 (H_d Sylvester Hadamard:
+ *                                                      H[j,i] = (-1)^popcount(i & j))
+ * and y is written to any subset of out [n, d] (out_dtype), out_kv (FP8/BF16 rows quantised as
+ * by csa_quantize_kv, out_kv->rope_dims giving the BF16 part) and out_fp4 (FP4 rows quantised as
+ * by csa_quantize_fp4).  fp32 arithmetic, rotation angles in fp64.  Limits: d one of 32, 64,
+ * 128, 256, 512; rd even, 0 <= rd <= d; base > 1 when rd > 0.
+ * Errors: CSA_ERR_INVALID_ARG for a null x, n < 0, a bad dtype, x or out not 16-byte aligned, rd
+ * odd or outside [0, d], rd > 0 without pos or with base <= 1, a g with a negative or non-finite
+ * eps, no output, or an output row struct that does not hold n rows of d; CSA_ERR_UNSUPPORTED for
+ * another d.
+ */
+int csa_prep_rows(const void *x, int32_t in_dtype, int64_t n, int32_t d, const float *g, float eps, int32_t rd,
+                  const int64_t *pos, double base, int32_t hadamard, void *out, int32_t out_dtype,
+                  const csa_kv_rows *out_kv, const csa_fp4_rows *out_fp4, void *stream);
+
 /* ----------------------------------------------------------------------------------------- */
 
 /*
@@ -184,24 +250,41 @@ int indexer_topk(const void *q, const float *w, const void *keys, int32_t fmt,
                  int32_t *idx_out, float *score_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * indexer_topk_paged -- indexer_topk (FP4 64 x 128 decode path) over paged index keys: entry s of
+ * query r is key row pages[r * max_pages + s / page_rows] * page_rows + s % page_rows of `keys`
+ * (a `const csa_fp4_rows*`), in place of key_off[r] + s; nv(r) = min(N_vis(q_pos[r]), max_nvis,
+ * max_pages * page_rows).  page_rows must be a power of two in [8, 128] (whole pages per 128-key
+ * tile).  A key whose page index or row is out of range gets score -inf and sets
+ * CSA_DEVERR_INDEX.  Workspace and results as for indexer_topk; CSA_ERR_UNSUPPORTED for any
+ * other shape or page size.
+ */
+int indexer_topk_paged(const void *q, const float *w, const void *keys, const int64_t *q_pos, int64_t Nq,
+                       int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis, const int32_t *pages,
+                       int32_t max_pages, int32_t page_rows, int32_t *idx_out, float *score_out, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/*
  * indexer_topk_static -- indexer_topk for callers that cannot allocate device memory (for
  * example runtimes that reserve the device memory for their own pools up front and give plugins
  * no allocator).  The pages have no counterpart: this is a library convenience.
  *
- * Same arguments, semantics and results as indexer_topk, without the workspace: the score
- * scratch is a file-scope device array of indexer_topk_static_capacity() = 4,194,304 fp32 scores
- * (16 MiB), which every GPU that loads this library holds until the process exits.  Requests
- * with Nq * ceil4(max_nvis) above that capacity return CSA_ERR_SCRATCH_CAPACITY before anything
- * is launched.  No cudaMalloc, cudaFree or allocating library routine is called.  An empty
- * batch (Nq = 0) is checked like any other and returns CSA_OK without touching the device.
+ * Same arguments, semantics, checks and results as indexer_topk, without the workspace: the
+ * scratch is a file-scope device array of indexer_topk_static_capacity() = 16 MiB + 256 bytes,
+ * which every GPU that loads this library holds until the process exits.  A request is refused
+ * with CSA_ERR_SCRATCH_CAPACITY, before anything is launched, when the scratch of the path it
+ * takes on this device does not fit: Nq * ceil4(max_nvis) * 4 bytes of scores (plus 256 of
+ * alignment) on every path, plus, on the FP4 64 x 128 decode path, the per-chunk candidate
+ * lists (at most Nq * 208,128 bytes; 12 sequences at 1M context fit, 16 do not).  No
+ * cudaMalloc, cudaFree or allocating library routine is called.  An empty batch (Nq = 0) is
+ * checked like any other and returns CSA_OK without touching the device.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  *     with that device current); make that first call before any stream capture begins.
  *   - All calls on a device share the one array, which keeps the last call's contents.  Nothing
- *     in it needs to start at zero (each call writes every score it reads), but calls whose
+ *     in it needs to start at zero (each call writes every value it reads), but calls whose
  *     kernels overlap on the GPU (different streams without ordering) race on it: serialise them.
  */
 #define CSA_ERR_SCRATCH_CAPACITY (-6) /* request exceeds the static scratch of *_static calls */
-size_t indexer_topk_static_capacity(void);
+size_t indexer_topk_static_capacity(void); /* bytes */
 int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t fmt,
                         const int64_t *q_pos, const int64_t *key_off, int64_t n_keys, int64_t Nq,
                         int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis,
@@ -221,8 +304,9 @@ int indexer_topk_static(const void *q, const float *w, const void *keys, int32_t
  *   o[t,h,:] = sum e^z key / (e^{sink[h]} + sum e^z),  lse[t,h] = ln(e^{sink[h]} + sum e^z).
  *
  *   q [T, H, c], x_win [T, c], kv_comp [n_comp, c] in `dtype` (CSA_F32 / CSA_BF16)
- *   idx [T, k] int32 or NULL; negative entries (padding) are skipped, entries >= n_comp are
- *            skipped and set CSA_DEVERR_INDEX
+ *   idx [T, k] int32 or NULL; negative entries (padding) are skipped; entries >= n_comp, and
+ *            entries >= N_vis(t) (a block the query is still inside), are skipped and set
+ *            CSA_DEVERR_INDEX
  *   sink [H] fp32 (-inf allowed: no sink);  o [T, H, c] in `dtype`;  lse [T, H] fp32 or NULL
  * Limits: c one of 32, 64, 128, 256, 512; 1 <= H <= 128; 1 <= W <= 1024; 0 <= k <= 4096.
  * Errors: CSA_ERR_INVALID_ARG for a null q, x_win, sink or o, T < 0, n_comp < 0, m < 1, a
@@ -244,7 +328,8 @@ int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, i
  *   win      window cache rows, sequence b's rows are b*W .. b*W + win_len[b] - 1, in any order
  *   win_len  [B] int32 in [0, W]
  *   idx      [B, k] int32 compressed-entry indices (CSA, -1 = empty) or NULL (HCA: all
- *            s < min(N_vis, max_nvis))
+ *            s < min(N_vis, max_nvis)); entries s >= min(N_vis, max_nvis) (not yet visible), or
+ *            whose row comp_off[b] + s lies outside comp, are skipped and set CSA_DEVERR_INDEX
  *   o        [B, H, c] bf16;  lse [B, H] fp32 or NULL
  *   ws       workspace of hybrid_attn_decode_workspace_size(...) bytes (split-K partials)
  * Limits: c one of 32, 64, 128, 256, 512; 1 <= H <= 128; 1 <= W <= 1024; 1 <= k <= 4096 with
@@ -255,6 +340,21 @@ int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, i
  * CSA_ERR_UNSUPPORTED for c, H, W or the key count outside the limits; CSA_ERR_WORKSPACE when
  * ws is NULL or smaller than the size above.
  */
+/*
+ * hybrid_attn_decode_paged -- hybrid_attn_decode over a paged compressed cache (the block-managed
+ * cache of [qa] Question 5; pages of page_rows entries, e.g. 32 CSA entries or 1 HCA entry for
+ * 128-token pages): entry s of sequence b is row pages[b * max_pages + s / page_rows] * page_rows
+ * + s % page_rows of comp, in place of comp_off[b] + s.  A page index >= max_pages or a row
+ * outside comp is skipped and sets CSA_DEVERR_INDEX.  Everything else, the workspace included,
+ * is as for hybrid_attn_decode; CSA_ERR_INVALID_ARG also for a null pages, max_pages < 1 or
+ * page_rows < 1.
+ */
+int hybrid_attn_decode_paged(const void *q, const csa_kv_rows *comp, const int32_t *pages, int32_t max_pages,
+                             int32_t page_rows, const int64_t *pos, const csa_kv_rows *win, const int32_t *win_len,
+                             const int32_t *idx, int32_t k, const float *sink, float scale, int32_t B, int32_t H,
+                             int32_t c, int32_t m, int32_t W, int64_t max_nvis, void *o, float *lse, void *ws,
+                             size_t ws_bytes, void *stream);
+
 size_t hybrid_attn_decode_workspace_size(int32_t B, int32_t H, int32_t c, int32_t k, int32_t W,
                                          int64_t max_nvis, int32_t use_idx);
 int hybrid_attn_decode(const void *q, const csa_kv_rows *comp, const int64_t *comp_off,
@@ -284,6 +384,37 @@ int csa_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int
                     void *q_next, const csa_fp4_rows *qI, void *stream);
 
 /* ----------------------------------------------------------------------------------------- */
+
+/*
+ * The kernel path that served the calling host thread's last indexer_topk(_static),
+ * hybrid_attn_prefill or hybrid_attn_decode call that launched work (CSA_PATH_NONE before any).
+ * Dispatch is by shape only: the tensor-core kernels take the 64-head x 512-channel attention
+ * and the 64 x 128 indexer shapes, the CUDA-core kernels every other shape the limits allow.
+ * A call whose shape belongs to a tensor-core kernel never moves to a CUDA-core one: if that
+ * kernel cannot be set up (e.g. no tensor-map encoder), the call returns CSA_ERR_CUDA.
+ */
+#define CSA_PATH_NONE 0
+#define CSA_PATH_INDEXER_FP4_TC 1   /* FP4 64 x 128: tcgen05 kind::mxf4 scan + threshold merge */
+#define CSA_PATH_INDEXER_BF16_TC 2  /* bf16 64 x 128 prefill: tcgen05 scores + per-query top-k */
+#define CSA_PATH_INDEXER_GENERIC 3  /* any other shape: CUDA-core scores + per-query top-k */
+#define CSA_PATH_PREFILL_TC 4       /* bf16 64 x 512, W = 128: tcgen05 attention */
+#define CSA_PATH_PREFILL_GENERIC 5
+#define CSA_PATH_DECODE_TC 6        /* 64 x 512: tcgen05 split-K attention + merge */
+#define CSA_PATH_DECODE_GENERIC 7
+#define CSA_PATH_PREFILL_PAIR_TC 8  /* bf16 64 x 512, W = 128, HCA: two tokens per item, 2-CTA cluster */
+int32_t csa_last_path(void);
+
+/*
+ * csa_set_wait_limit_ns -- how long the bounded waits of hybrid_attn_decode's tensor-core kernel
+ * may wait before they give up (record CSA_DEVERR_TIMEOUT and wind the CTA down), in ns, for the
+ * calls launched after it (process-wide); 0 restores the default of 2 s.  Returns the previous
+ * limit.  A limit of 1 ns turns every such wait into one non-blocking test that gives up unless
+ * its phase has already completed.  The pages have no counterpart: this exists so that a test can
+ * make the waits run out on purpose and check that the kernel winds down cleanly (it copies
+ * nothing asynchronously into shared memory, and its final drain of its own MMAs always allows
+ * the full 2 s) and that the next call is correct.
+ */
+uint64_t csa_set_wait_limit_ns(uint64_t ns);
 
 /* Synchronise `stream`, return the device error word (CSA_DEVERR_* bits) in *out and clear it. */
 int csa_device_error(void *stream, int32_t *out);

@@ -34,7 +34,8 @@ int main(void)
     csa_fp4_rows k4 = {(uint8_t *)f, (uint8_t *)f, 1000, 128};
     int status;
 
-    EXPECT(csa_abi_version(), 100);
+    EXPECT(csa_abi_version(), 101);
+    EXPECT(csa_last_path(), CSA_PATH_NONE);
     for (status = 0; status >= -6; status--) {
         const char *s = csa_status_string(status);
         if (!s || !s[0]) {
@@ -44,7 +45,7 @@ int main(void)
     }
     EXPECT(indexer_topk_workspace_size(10, 7, 4) >= 10 * 8 * 4, 1);
     EXPECT(hybrid_attn_decode_workspace_size(2, 64, 512, 1024, 128, 262144, 1) > 0, 1);
-    EXPECT(indexer_topk_static_capacity(), 4194304);
+    EXPECT(indexer_topk_static_capacity(), (16 << 20) + 256);
 
     /* bad arguments */
     EXPECT(csa_compress(NULL, f, f, f, ff, 8, 16, 4, CSA_F32, f, CSA_F32, NULL, NULL, NULL), CSA_ERR_INVALID_ARG);

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(C):
 
 
 def test_status_strings_and_version(C):
-    assert C.csa_abi_version() == 100
+    assert C.csa_abi_version() == 101
     assert C.status_string(0) == "ok"
     assert "workspace" in C.status_string(C.CSA_ERR_WORKSPACE)
 

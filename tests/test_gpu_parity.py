@@ -165,6 +165,7 @@ def test_indexer_topk_bf16_multi_tile(C):
     wt = WL.draw(w, "w", 0, T)
     idx_o, S = O.indexer_topk(q, wt, K, rows, m, k)
     idx = C.indexer_topk(dev(q, "bf16"), dev(wt), dev(K, "bf16"), m, k, max_nvis=T // m)
+    assert C.csa_last_path() == C.CSA_PATH_INDEXER_BF16_TC
     assert check_topk(idx.cpu().numpy(), idx_o, S, O.n_vis(rows, m), k) >= T - 8
 
 
@@ -189,6 +190,7 @@ def test_indexer_topk_fp4_decode_batches(C):
     C.csa_quantize_fp4(dev(qx.reshape(Bn * H, d)), q4)
     idx = C.indexer_topk(q4, dev(wt), k4, m, k, max_nvis=int(nv.max()),
                          q_pos=torch.from_numpy(pos).cuda(), key_off=torch.from_numpy(off).cuda())
+    assert C.csa_last_path() == C.CSA_PATH_INDEXER_FP4_TC
     assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
 
 
@@ -244,6 +246,47 @@ def test_fp4_decode_topk_ties_across_chunks(C, Bn, n0):
         assert list(ig[b]) == list(range(k))
     assert list(ig[Bn - 1]) == list(range(700)) + [-1] * (k - 700)
     assert np.all(sc.cpu().numpy()[idx.cpu().numpy() >= 0] == 0.0)
+
+
+@pytest.mark.parametrize("Bn", [2, 8])
+def test_fp4_decode_saturated_chunk(C, Bn):
+    """Keys of the last 12,000 entries of each sequence scaled by 4, so nearly all of the top-k
+    falls into the last chunk of the scan: that chunk holds far more than its share, its
+    published list cannot cover the winners, and the merge re-reads its stored scores.  Exact
+    against the oracle up to the 1e-4 tie band."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    H, d, m, k = 64, 128, 4, 1024
+    nv = np.array([90000 + 1000 * b for b in range(Bn)], np.int64)
+    pos = nv * m + 1
+    off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+    parts = []
+    for b, n in enumerate(nv):
+        x = WL.draw(w, "KI", 0, int(n), seq=300 + b)
+        x[-12000:] *= 4.0
+        parts.append(x)
+    keys = np.concatenate(parts)
+    qx = np.stack([WL.draw(w, "qI", 0, 1, seq=300 + b).reshape(H, d) for b in range(Bn)])
+    wt = np.concatenate([WL.draw(w, "w", 0, 1, seq=300 + b) for b in range(Bn)])
+    kc, ks = O.quant_fp4(keys)
+    qc, qs = O.quant_fp4(qx.reshape(Bn * H, d))
+    idx_o, S = O.indexer_topk(O.dequant_fp4(qc, qs).reshape(Bn, H, d), wt, O.dequant_fp4(kc, ks), pos, m, k, kbase=off)
+    assert (idx_o >= nv[:, None] - 12000).mean() > 0.9   # the winners sit in the scaled tail
+    k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
+    q4 = C.Fp4Rows.empty(Bn * H, d, "cuda")
+    C.csa_quantize_fp4(dev(keys), k4)
+    C.csa_quantize_fp4(dev(qx.reshape(Bn * H, d)), q4)
+    sc = torch.empty((Bn, k), dtype=torch.float32, device="cuda")
+    idx = C.indexer_topk(q4, dev(wt), k4, m, k, max_nvis=int(nv.max()), q_pos=torch.from_numpy(pos).cuda(),
+                         key_off=torch.from_numpy(off).cuda(), score_out=sc)
+    torch.cuda.synchronize()
+    assert C.csa_last_path() == C.CSA_PATH_INDEXER_FP4_TC
+    assert C.csa_device_error() == 0
+    ig = idx.cpu().numpy()
+    assert check_topk(ig, idx_o, S, nv, k) >= Bn - 1
+    for b in range(Bn):  # scores of the selected entries, descending
+        sb = sc.cpu().numpy()[b]
+        assert np.all(np.diff(sb) <= 0)
+        np.testing.assert_allclose(sb, S[b, ig[b]], rtol=1e-4, atol=1e-5)
 
 
 def test_topk_ties_short_lists_and_scores(C):
@@ -302,11 +345,15 @@ def test_prefill_attention_hca_bf16(C, T, W, m):
     np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
 
 
-@pytest.mark.parametrize("T,m,k", [(1, 4, None), (130, 128, None), (2000, 16, None), (300, 4, 512), (157, 4, 200)])
+@pytest.mark.parametrize("T,m,k", [(1, 4, None), (2, 4, None), (77, 4, None), (130, 128, None), (257, 64, None),
+                                   (300, 16, None), (2000, 16, None), (300, 4, 512), (157, 4, 200)])
 def test_prefill_attention_tensor_core_shapes(C, T, m, k):
-    """64 heads x 512 channels, bf16, window 128: the tcgen05 path.  Covers a single token, fewer
-    tokens than SMs, several tokens per CTA, 1-2 compressed tiles, 4 top-k tiles with many empty
-    (-1) slots and a top-k length that is not a multiple of the 128-key tile."""
+    """64 heads x 512 channels, bf16, window 128: the tcgen05 paths.  HCA (all visible entries)
+    runs two tokens per item on a 2-CTA cluster: a single token, a single pair, an odd token count
+    (the last item has one token), block boundaries between the two tokens of a pair (m = 4, 16,
+    64, 128), fewer pairs than clusters and several per cluster.  CSA (top-k lists) runs one token
+    per pass: 4 top-k tiles with many empty (-1) slots and a length that is not a multiple of the
+    128-key tile."""
     w = _wl("csa_prefill_64k", T=T, m=m)
     n_comp = max(T // m, 1)
     q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
@@ -315,6 +362,7 @@ def test_prefill_attention_tensor_core_shapes(C, T, m, k):
     lse = torch.empty((T, 64), dtype=torch.float32, device="cuda")
     o = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, 128,
                               idx=None if idx is None else dev_i(idx), lse=lse)
+    assert C.csa_last_path() == (C.CSA_PATH_PREFILL_PAIR_TC if k is None else C.CSA_PATH_PREFILL_TC)
     err = row_rel_err(host(o), o_ref)
     assert err.max() < 2e-2, err.max()
     np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
@@ -339,6 +387,15 @@ def test_prefill_attention_csa_bf16_with_invalid_indices(C):
     o2 = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, w.W, idx=dev_i(bad))
     assert C.csa_device_error() & C.CSA_DEVERR_INDEX
     assert row_rel_err(host(o2)[5], o_ref2[0]).max() < 2e-2
+    # an entry of the block the query is still inside (token 605 sees entries < 151): skipped, reported
+    bad2 = idx.copy()
+    bad2[605, 3] = 151
+    ref3 = bad2.copy()
+    ref3[605, 3] = -1
+    o_ref3, _ = O.hybrid_attn_prefill(q, X, KVc, sink, 1.0, m, w.W, idx=ref3, rows=[605])
+    o3 = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, w.W, idx=dev_i(bad2))
+    assert C.csa_device_error() & C.CSA_DEVERR_INDEX
+    assert row_rel_err(host(o3)[605], o_ref3[0]).max() < 2e-2
 
 
 # ---------------------------------------------------------------------------------------------
@@ -374,9 +431,23 @@ def test_decode_attention_mixed_cache(C, use_idx):
     o = C.hybrid_attn_decode(dev(WL.on_grid(q, "bf16"), "bf16"), ckv, torch.from_numpy(off).cuda(),
                              torch.from_numpy(pos).cuda(), wkv, dev_i(win_len), dev(sink), 1.0, m, W,
                              max_nvis=int(nv.max()), idx=None if idx is None else dev_i(idx), lse=lse)
+    assert C.csa_last_path() == C.CSA_PATH_DECODE_TC
     assert row_rel_err(host(o), o_ref).max() < 2e-2
     # the tensor-core path rounds dequantised FP8 keys to bf16 (2^-9 relative) before the MMA
     np.testing.assert_allclose(host(lse), lse_ref, atol=1e-2)
+    assert C.csa_device_error() == 0
+    if use_idx:  # an entry sequence 2 cannot see yet (its token at 129 sees entries < 32): skipped, reported
+        bad = idx.copy()
+        bad[2, 5] = int(nv[2])
+        ref = bad.copy()
+        ref[2, 5] = -1
+        o_ref2, _ = O.hybrid_attn_decode(WL.on_grid(q, "bf16"), O.dequant_kv(cf, cr, cs), off, pos,
+                                         O.dequant_kv(wf, wr, ws), win_len, sink, 1.0, m, W, idx=ref)
+        o2 = C.hybrid_attn_decode(dev(WL.on_grid(q, "bf16"), "bf16"), ckv, torch.from_numpy(off).cuda(),
+                                  torch.from_numpy(pos).cuda(), wkv, dev_i(win_len), dev(sink), 1.0, m, W,
+                                  max_nvis=int(nv.max()), idx=dev_i(bad))
+        assert C.csa_device_error() & C.CSA_DEVERR_INDEX
+        assert row_rel_err(host(o2), o_ref2).max() < 2e-2
 
 
 def test_decode_attention_multi_tile_items(C):

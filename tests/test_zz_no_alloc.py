@@ -71,9 +71,29 @@ def test_static_scratch_matches_workspace_entry_point_twice_in_a_row(C):
 
 def test_static_scratch_rejects_requests_beyond_capacity(C):
     cap = int(C.lib().indexer_topk_static_capacity())
-    assert cap == 4 << 20
+    assert cap == (16 << 20) + 256
     f = ctypes.c_void_p(0x100000)  # never dereferenced: the size check comes first
-    st = C.lib().indexer_topk_static(f, f, f, C.CSA_BF16, None, None, 1 << 22, 17, 8, 64, 4, 16, cap // 16,
+    st = C.lib().indexer_topk_static(f, f, f, C.CSA_BF16, None, None, 1 << 22, 17, 8, 64, 4, 16, cap // 64,
                                      f, None, None)
     assert st == C.CSA_ERR_SCRATCH_CAPACITY
     assert "static scratch" in C.status_string(st)
+
+
+def test_static_scratch_capacity_counts_the_decode_lists(C):
+    """On the FP4 64 x 128 decode path the scratch holds the chunk candidate lists next to the
+    scores: 16 sequences at 1M context (262,144 entries each) fill the array with their scores
+    alone, so the lists tip them over; 12 sequences fit.  Nothing is launched: the capacity check
+    comes first, and the accepted request then fails the row check (its query rows are short)."""
+    lib = C.lib()
+    f = ctypes.c_void_p(0x100000)
+    nv = 262144
+
+    def call(nq, q_rows):
+        q4 = C._Fp4Rows(0x100000, 0x100000, q_rows, 128)
+        k4 = C._Fp4Rows(0x100000, 0x100000, nq * nv, 128)
+        return lib.indexer_topk_static(ctypes.byref(q4), f, ctypes.byref(k4), C.CSA_FP4, None, None, nq * nv, nq,
+                                       64, 128, 4, 1024, nv, f, None, None)
+
+    assert 16 * nv * 4 + 256 <= lib.indexer_topk_static_capacity()  # the scores alone would fit
+    assert call(16, 16 * 64) == C.CSA_ERR_SCRATCH_CAPACITY
+    assert call(12, 1) == C.CSA_ERR_INVALID_ARG  # past the capacity check, stopped by the row check
