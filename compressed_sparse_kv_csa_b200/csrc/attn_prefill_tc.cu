@@ -75,7 +75,7 @@ __device__ __forceinline__ int n_tiles(int64_t n_cmp) { return 1 + (int)((n_cmp 
 
 // Key row of slot j of tile i for token t, or nullptr when the slot is empty.
 __device__ __forceinline__ const uint16_t *key_row(const PrefillArgs &a, int64_t t, int i, int j, int64_t n_cmp,
-                                                   bool report)
+                                                   int64_t nvt, bool report)
 {
     if (i == 0) {
         const int64_t u = t - (kW - 1) + j;
@@ -85,7 +85,7 @@ __device__ __forceinline__ const uint16_t *key_row(const PrefillArgs &a, int64_t
     if (slot >= n_cmp) return nullptr;
     const int64_t s = a.idx ? (int64_t)a.idx[t * a.k + slot] : slot;
     if (s < 0) return nullptr;
-    if (s >= a.n_comp || s >= (t + 1) / a.m) { // missing, or not yet visible to t
+    if (s >= a.n_comp || s >= nvt) { // missing, or not yet visible to t (nvt = N_vis(t))
         if (report) flag_error(a.err, CSA_DEVERR_INDEX);
         return nullptr;
     }
@@ -128,12 +128,12 @@ struct TmaMaps {
 
 // Compressed row of slot j of CSA tile i for token t, or -1 when the slot is empty or invalid.
 __device__ __forceinline__ int32_t gather_row(const PrefillArgs &a, int64_t t, int i, int j, int64_t n_cmp,
-                                              bool report)
+                                              int64_t nvt, bool report)
 {
     const int64_t slot = (int64_t)(i - 1) * kKT + j;
     if (slot >= n_cmp) return -1;
     const int32_t s = a.idx[t * a.k + slot];
-    if (s >= a.n_comp || s >= (t + 1) / a.m) { // missing, or not yet visible to t
+    if (s >= a.n_comp || s >= nvt) { // missing, or not yet visible to t (nvt = N_vis(t))
         if (report) flag_error(a.err, CSA_DEVERR_INDEX);
         return -1;
     }
@@ -163,6 +163,7 @@ __device__ __forceinline__ bool softmax_role(const PrefillArgs &a, const Smem &S
     uint32_t s_ph = 0, pv_ph = 0;
     for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
         const int64_t n_cmp = n_compressed(a, t);
+        const int64_t nvt = (t + 1) / a.m; // N_vis(t), once per token
         const int nt = n_tiles(n_cmp);
         float m_run = -INFINITY, l_run = 0.f;
         for (int i = 0; i < nt; ++i) {
@@ -188,7 +189,7 @@ __device__ __forceinline__ bool softmax_role(const PrefillArgs &a, const Smem &S
             uint32_t vm[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                vm[q] = __ballot_sync(0xffffffffu, key_row(a, t, i, lane + 32 * q, n_cmp, false) != nullptr);
+                vm[q] = __ballot_sync(0xffffffffu, key_row(a, t, i, lane + 32 * q, n_cmp, nvt, false) != nullptr);
             const uint32_t m0 = upper ? vm[0] : vm[2], m1 = upper ? vm[1] : vm[3];
             float mt = -INFINITY;
 #pragma unroll
@@ -294,6 +295,7 @@ __device__ __forceinline__ bool producer_role(const PrefillArgs &a, const TmaMap
     bool first_q = true, first_h[2] = {true, true};
     for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
         const int64_t n_cmp = n_compressed(a, t);
+        const int64_t nvt = (t + 1) / a.m; // N_vis(t), once per token
         const int nt = n_tiles(n_cmp);
         if (ptid == 0) { // Q [64 rows x 512] = 8 boxes of 64 x 64
             if (!first_q) {
@@ -334,7 +336,7 @@ __device__ __forceinline__ bool producer_role(const PrefillArgs &a, const TmaMap
                 int32_t rr[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int32_t s = gather_row(a, t, i, 4 * g + u, n_cmp, h == 0 && q == 0);
+                    const int32_t s = gather_row(a, t, i, 4 * g + u, n_cmp, nvt, h == 0 && q == 0);
                     rr[u] = s < 0 ? 0 : s;
                 }
                 mbar_arrive_expect_tx(S.bar(B_KVFULL0 + h), 512u);
@@ -352,6 +354,7 @@ __device__ __forceinline__ bool mma_role(const PrefillArgs &a, const Smem &S, ui
     uint32_t q_ph = 0, kf_ph[2] = {0, 0}, p_ph = 0;
     for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
         const int64_t n_cmp = n_compressed(a, t);
+        const int64_t nvt = (t + 1) / a.m; // N_vis(t), once per token
         const int nt = n_tiles(n_cmp);
         if (!mbar_wait(S.bar(B_QFULL), q_ph)) return false;
         q_ph ^= 1;

@@ -48,8 +48,9 @@ using namespace tc;
 
 constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 8;
 constexpr int kChunk = 16384;                 // most keys per CTA
-constexpr int kR = 8;                         // keys kept per epilogue thread
+constexpr int kR = 16;                        // keys kept per epilogue thread
 constexpr int kMergeSmem = 200 * 1024;        // merge kernel: published lists + winners
+constexpr int kShareMax = 512;                // most of k one chunk is expected to hold
 constexpr int kProdWarp = 0, kEpiWarp0 = 1, kEpiWarps = 8, kMmaWarp = kEpiWarp0 + kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -101,6 +102,27 @@ __device__ __forceinline__ int64_t dec_nvis(const IndexerArgs &a, int64_t r)
     return nv < 0 ? 0 : nv;
 }
 
+// Query r's chunk size: its nv visible keys spread over all n_slots chunks (multiples of the
+// 128-key tile), so every query's chunks hold about the same share of its k winners.
+__host__ __device__ __forceinline__ int query_chunk(int64_t nv, int n_slots)
+{
+    int64_t ch = (nv + n_slots - 1) / n_slots;
+    ch = (ch + kKT - 1) / kKT * kKT;
+    return (int)(ch < kKT ? kKT : ch);
+}
+
+// Keys a chunk of query r publishes: about twice its share of k (at least 64), at most the list
+// capacity and at most k.
+__host__ __device__ __forceinline__ int query_keep(int64_t nv, int chunk, int k, int lcap)
+{
+    const int64_t ns = nv > 0 ? (nv + chunk - 1) / chunk : 1;
+    const int64_t share = (k + ns - 1) / ns;
+    int64_t keep = 2 * share + 32;
+    keep = keep < 64 ? 64 : keep;
+    keep = keep > k ? k : keep;
+    return (int)(keep > lcap ? lcap : keep);
+}
+
 __device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity)
 {
     const bool ok = mbar_wait(bar, parity);
@@ -119,7 +141,7 @@ struct ChunkOut {
     unsigned long long *list;   // [Nq, n_slots, lcap]
     int *count;                 // [Nq, n_slots]
     unsigned long long *theta;  // [Nq, n_slots]
-    int n_slots, chunk, lcap, keep;
+    int n_slots, lcap;
 };
 
 __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
@@ -156,8 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t r = blockIdx.y;
     const int slot = blockIdx.x;
-    const int chunk = co.chunk;
     const int64_t nv = dec_nvis(a, r);
+    const int chunk = query_chunk(nv, co.n_slots);
+    const int keep = query_keep(nv, chunk, a.k, co.lcap);
     const int64_t c0 = (int64_t)slot * chunk;
     const int n = (int)(nv - c0 < chunk ? (nv - c0 > 0 ? nv - c0 : 0) : chunk);
     const int64_t oslot = r * co.n_slots + slot;
@@ -311,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const int nu = misc[M_COUNT];
             unsigned long long theta_c = tau;
             int cnt;
-            if (nu <= co.keep) { // publish everything
+            if (nu <= keep) { // publish everything
                 for (int j = etid; j < nu; j += kEpiThreads) out[j] = U[j];
                 cnt = nu;
             } else {
@@ -320,10 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
                 uint32_t kmin;
                 int lead, n_ge;
                 const int bin = top_bin32<kEpiThreads, kEpiBar>(
-                    nu, co.keep, [&](int j) { return (uint32_t)(U[j] >> 32); }, sel, kmin, lead, n_ge, etid);
+                    nu, keep, [&](int j) { return (uint32_t)(U[j] >> 32); }, sel, kmin, lead, n_ge, etid);
                 unsigned long long thr = 0ull;
                 if (n_ge > co.lcap)
-                    thr = block_kth64<kEpiThreads, kEpiBar>(nu, co.keep, [&](int j) { return U[j]; }, sel, etid);
+                    thr = block_kth64<kEpiThreads, kEpiBar>(nu, keep, [&](int j) { return U[j]; }, sel, etid);
                 unsigned long long mx = 0ull; // the largest key that is not published
                 for (int j = etid; j < nu; j += kEpiThreads) {
                     const unsigned long long v = U[j];
@@ -392,8 +415,9 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a
     __shared__ unsigned long long s_theta[kMaxSlots];
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
-    const int k = a.k, ns = co.n_slots, chunk = co.chunk;
+    const int k = a.k, ns = co.n_slots;
     const int64_t nv = dec_nvis(a, r);
+    const int chunk = query_chunk(nv, ns);
     if (tid == 0) {
         int o = 0;
         for (int sl = 0; sl < ns; ++sl) {
@@ -511,32 +535,31 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a
     }
 }
 
-// Chunking of the key lists: at most one CTA per SM (the CTAs of one launch fill a single wave),
-// at most kChunk keys each; each chunk publishes `keep` keys (about twice its share of k, at
-// least 64) in a list of lcap slots sized so the merge holds every list in shared memory.
+// Chunking of the key lists: each query's keys are spread over n_slots chunks (query_chunk),
+// enough that a chunk's expected share of k is at most kShareMax and that the launch fills the
+// SMs; a chunk holds at most kChunk keys.  Every chunk publishes into a list of lcap slots, sized
+// so that the merge holds all of a query's lists in shared memory.
 struct Plan {
-    int slots, chunk, keep, lcap;
+    int slots, lcap;
 };
 
 bool scan_plan(int64_t Nq, int64_t max_nvis, int k, int sms, Plan *p)
 {
     int64_t want = sms / (Nq > 0 ? Nq : 1);
+    const int64_t by_share = (k + kShareMax - 1) / kShareMax;
+    if (want < by_share) want = by_share;
     if (want < 1) want = 1;
     int64_t ch = (max_nvis + want - 1) / want;
     ch = (ch + kKT - 1) / kKT * kKT;
     if (ch > kChunk) ch = kChunk;
     if (ch < kKT) ch = kKT;
-    p->chunk = (int)ch;
     p->slots = (int)((max_nvis + ch - 1) / ch);
     if (p->slots < 1) p->slots = 1;
-    const int share = (k + p->slots - 1) / p->slots;
-    p->keep = 2 * share + 32 > 64 ? 2 * share + 32 : 64;
-    if (p->keep > k) p->keep = k;
     int n2 = 1;
     while (n2 < k) n2 <<= 1;
     const int64_t room = (kMergeSmem - (int64_t)n2 * 8) / ((int64_t)p->slots * 8);
-    p->lcap = (int)(room < 512 ? room : 512);
-    return p->slots <= kMaxSlots && p->lcap >= p->keep;
+    p->lcap = (int)(room < kEpiThreads * kR ? room : kEpiThreads * kR);
+    return p->slots <= kMaxSlots && p->lcap >= query_keep(max_nvis, query_chunk(max_nvis, p->slots), k, 1 << 30);
 }
 
 size_t lists_bytes(int64_t Nq, const Plan &p)
@@ -584,9 +607,7 @@ cudaError_t launch_indexer_decode(const IndexerArgs &a0, void *ws, cudaStream_t 
     co.theta = co.list + (size_t)a0.Nq * p.slots * p.lcap;
     co.count = reinterpret_cast<int *>(co.theta + (size_t)a0.Nq * p.slots);
     co.n_slots = p.slots;
-    co.chunk = p.chunk;
     co.lcap = p.lcap;
-    co.keep = p.keep;
     IndexerArgs a = a0;
     a.scores = reinterpret_cast<float *>(base + lists_bytes(a0.Nq, p));
     a.ld = (a0.max_nvis + 3) / 4 * 4;

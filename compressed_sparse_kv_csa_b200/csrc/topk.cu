@@ -5,11 +5,14 @@
 // convention of this library: score descending, equal scores by lower entry index; unused slots
 // hold -1.
 //
-// One CTA per query row.  Radix select over order-preserving 32-bit keys of the fp32 scores
-// (8-bit digits over the bits that differ within the row, select.cuh) finds the exact k-th key; entries
-// above it are taken unordered, entries equal to it are collected and the lowest-index ones kept
-// (a second selection over the tie list), and the k_eff winners are then sorted in shared memory (bitonic, 64-bit keys
-// (score key, inverted index)).
+// One CTA of 512 threads per query row; rows of at most TK_STAGE scores are staged in shared
+// memory as order-preserving 32-bit keys.  Every entry has the unique 64-bit key
+// (score key << 32 | ~index), so "the k largest keys" is exactly the wanted set.  Three passes
+// over the row: (1) the range of the score keys; (2) a histogram of the top 11 bits of the keys
+// offset by the minimum and left-aligned on the range (2,048 bins, warp-aggregated atomics), whose
+// suffix sums give the bin b* that holds the k-th key; (3) keys in bins above b* are winners,
+// keys in b* are candidates (warp-aggregated appends).  The few candidates are resolved by an
+// exact 64-bit selection, and the k winners are sorted in shared memory (bitonic).
 #include "common.cuh"
 #include "select.cuh"
 
@@ -17,9 +20,11 @@ namespace csa {
 
 namespace {
 
-constexpr int TK_THREADS = 1024;
-constexpr int TK_MAX = 2048;
-constexpr int64_t TK_STAGE = 32768; // rows of at most this many scores are staged in shared memory
+constexpr int TK_THREADS = 512;
+constexpr int TK_MAX = 2048;     // largest k
+constexpr int TK_BINS = 2048;    // 11-bit first digit
+constexpr int TK_CAND = 2048;    // candidates of the crossing bin kept in shared memory
+constexpr int64_t TK_STAGE = 16384; // rows of at most this many scores are staged in shared memory
 
 __device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
 {
@@ -32,19 +37,38 @@ __device__ __forceinline__ int64_t tk_nvis(const IndexerArgs &a, int64_t r)
     return nv < 0 ? 0 : nv;
 }
 
-// STAGED: the row's scores (nv <= TK_STAGE) are first copied into shared memory as keys, so the
-// selection passes read shared memory instead of the score buffer.
+__device__ __forceinline__ unsigned long long key64(uint32_t k, int64_t i)
+{
+    return ((unsigned long long)k << 32) | (unsigned long long)(0xffffffffu - (uint32_t)i);
+}
+
+// Warp-aggregated append of the lanes with `take` to list[*count ...]; returns nothing.
+__device__ __forceinline__ void warp_append(bool take, unsigned long long v, unsigned long long *list, int *count,
+                                            int cap)
+{
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (!m) return;
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    if (lane == __ffs(m) - 1) base = atomicAdd(count, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+    const int p = base + __popc(m & ((1u << lane) - 1u));
+    if (take && p < cap) list[p] = v;
+}
+
 template <bool STAGED>
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
 {
     __shared__ unsigned long long sel[TK_MAX];
+    __shared__ unsigned long long cand[TK_CAND];
+    __shared__ int hist[TK_BINS];
     __shared__ SelectSmem<uint32_t> ssel;
-    __shared__ uint32_t ties[TK_MAX];
-    __shared__ int s_cnt, s_eq, s_warp[TK_THREADS / 32], s_eq_taken;
+    __shared__ uint32_t s_lo[TK_THREADS / 32], s_hi[TK_THREADS / 32];
+    __shared__ int s_bin, s_above, s_nsel, s_ncand;
     extern __shared__ uint32_t skeys[]; // STAGED only
 
     const int64_t r = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t nv = tk_nvis(a, r);
     const int k = a.k;
     const int ke = (int)(nv < k ? nv : k);
@@ -57,68 +81,107 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
             skeys[4 * i4 + 2] = float_key(v.z);
             skeys[4 * i4 + 3] = float_key(v.w);
         }
-        __syncthreads();
     }
-    auto key = [&](int64_t i) { return STAGED ? skeys[i] : float_key(S[i]); };
+    if (tid == 0) {
+        s_nsel = 0;
+        s_ncand = 0;
+    }
+    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0;
+    __syncthreads();
+    auto key = [&](int64_t i) -> uint32_t { return STAGED ? skeys[i] : float_key(S[i]); };
 
-    uint32_t thr = 0;   // k-th largest key (only meaningful when nv > k)
-    int n_gt = 0;       // number of keys strictly above thr
-    if (nv > k) {
-        block_kth<TK_THREADS, uint32_t>((int)nv, k, [&](int i) { return key(i); }, &ssel, thr, n_gt);
-        const int need = k - n_gt; // entries equal to the threshold that are taken: the lowest indices
-        if (tid == 0) { s_cnt = 0; s_eq = 0; s_eq_taken = 0; }
-        __syncthreads();
-        // strictly greater: unordered append; equal: their indices into the tie list
-        for (int64_t s = tid; s < nv; s += TK_THREADS) {
-            const uint32_t kv = key(s);
-            if (kv > thr) {
-                const int pos = atomicAdd(&s_cnt, 1);
-                if (pos < n_gt) sel[pos] = ((unsigned long long)kv << 32) | (0xffffffffu - (uint32_t)s);
-            } else if (kv == thr) {
-                const int e = atomicAdd(&s_eq, 1);
-                if (e < TK_MAX) ties[e] = (uint32_t)s;
-            }
-        }
-        __syncthreads();
-        const int n_eq = s_eq; // >= need
-        const unsigned long long hi = (unsigned long long)thr << 32;
-        if (n_eq <= TK_MAX) {
-            uint32_t lim = 0; // take the ties whose inverted index is >= lim
-            if (n_eq > need) {
-                int g;
-                block_kth<TK_THREADS, uint32_t>(n_eq, need, [&](int e) { return 0xffffffffu - ties[e]; }, &ssel, lim, g);
-            }
-            if (tid == 0) s_cnt = 0;
-            __syncthreads();
-            for (int e = tid; e < n_eq; e += TK_THREADS) {
-                const uint32_t inv = 0xffffffffu - ties[e];
-                if (inv >= lim) sel[n_gt + atomicAdd(&s_cnt, 1)] = hi | inv;
-            }
-        } else { // more ties than the list holds: ordered block scan from the lowest index
-            for (int64_t base = 0; base < nv; base += TK_THREADS) {
-                if (s_eq_taken >= need) break; // uniform: read after a barrier
-                const int64_t s = base + tid;
-                const bool eq = (s < nv) && (key(s) == thr);
-                const unsigned bal = __ballot_sync(0xffffffffu, eq);
-                const int lane = tid & 31, wid = tid >> 5;
-                if (lane == 0) s_warp[wid] = __popc(bal);
-                __syncthreads();
-                int before = 0, total = 0;
-                for (int w = 0; w < TK_THREADS / 32; ++w) {
-                    if (w < wid) before += s_warp[w];
-                    total += s_warp[w];
-                }
-                const int rank = s_eq_taken + before + __popc(bal & ((1u << lane) - 1u));
-                if (eq && rank < need) sel[n_gt + rank] = hi | (0xffffffffu - (uint32_t)s);
-                __syncthreads();
-                if (tid == 0) s_eq_taken += total;
-                __syncthreads();
-            }
-        }
+    if (nv <= k) { // every visible entry is a winner
+        for (int64_t i = tid; i < nv; i += TK_THREADS) sel[i] = key64(key(i), i);
     } else {
-        for (int64_t s = tid; s < nv; s += TK_THREADS)
-            sel[s] = ((unsigned long long)key(s) << 32) | (0xffffffffu - (uint32_t)s);
+        // 1. range of the score keys
+        uint32_t lo = 0xffffffffu, hi = 0;
+        for (int64_t i = tid; i < nv; i += TK_THREADS) {
+            const uint32_t v = key(i);
+            lo = v < lo ? v : lo;
+            hi = v > hi ? v : hi;
+        }
+        lo = warp_min_key(lo);
+        hi = warp_max_key(hi);
+        if (lane == 0) {
+            s_lo[wid] = lo;
+            s_hi[wid] = hi;
+        }
+        __syncthreads();
+        lo = s_lo[0];
+        hi = s_hi[0];
+        for (int w = 1; w < TK_THREADS / 32; ++w) {
+            lo = s_lo[w] < lo ? s_lo[w] : lo;
+            hi = s_hi[w] > hi ? s_hi[w] : hi;
+        }
+        const int lead = (hi == lo) ? 32 : __clz(hi - lo);
+        auto bin_of = [&](uint32_t v) -> int { return lead >= 32 ? 0 : (int)(((v - lo) << lead) >> 21); };
+        // 2. histogram of the 11-bit first digit (lanes with the same bin add once)
+        for (int64_t base = 0; base < nv; base += TK_THREADS) {
+            const int64_t i = base + tid;
+            const bool in = i < nv;
+            const int b = in ? bin_of(key(i)) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, b);
+            if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[b], __popc(peers));
+        }
+        __syncthreads();
+        if (wid == 0) { // suffix scan from the top bin: lane l owns bins 2047-64l .. 1984-64l
+            int sum = 0;
+            for (int j = 0; j < 64; ++j) sum += hist[TK_BINS - 1 - 64 * lane - j];
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int excl = incl - sum;
+            const bool cross = excl < k && incl >= k;
+            const unsigned who = __ballot_sync(0xffffffffu, cross);
+            if (cross && lane == __ffs(who) - 1) {
+                int cum = excl, j = 0;
+                for (; j < 63; ++j) {
+                    const int c = hist[TK_BINS - 1 - 64 * lane - j];
+                    if (cum + c >= k) break;
+                    cum += c;
+                }
+                s_bin = TK_BINS - 1 - 64 * lane - j;
+                s_above = cum; // keys in the bins above b*
+            }
+        }
+        __syncthreads();
+        const int bstar = s_bin, n_above = s_above, need = k - n_above;
+        // 3. winners above b*, candidates in b*
+        for (int64_t base = 0; base < nv; base += TK_THREADS) {
+            const int64_t i = base + tid;
+            const bool in = i < nv;
+            const uint32_t v = in ? key(i) : 0u;
+            const int b = in ? bin_of(v) : -1;
+            warp_append(in && b > bstar, key64(v, i), sel, &s_nsel, TK_MAX);
+            warp_append(in && b == bstar, key64(v, i), cand, &s_ncand, TK_CAND);
+        }
+        __syncthreads();
+        const int n_cand = s_ncand; // >= need
+        // 4. the `need` largest candidates join the winners
+        if (n_cand <= TK_CAND) {
+            const unsigned long long thr =
+                n_cand > need ? block_kth64<TK_THREADS>(n_cand, need, [&](int j) { return cand[j]; }, &ssel) : 0ull;
+            for (int j = tid; j < n_cand; j += TK_THREADS) {
+                const unsigned long long v = cand[j];
+                if (v >= thr) sel[atomicAdd(&s_nsel, 1)] = v; // s_nsel starts at n_above here
+            }
+        } else { // more candidates than shared memory holds (many equal scores): select over the row
+            auto get = [&](int j) -> unsigned long long {
+                const uint32_t v = key(j);
+                return bin_of(v) == bstar ? key64(v, j) : 0ull;
+            };
+            const unsigned long long thr = block_kth64<TK_THREADS>((int)nv, need, get, &ssel);
+            for (int64_t base = 0; base < nv; base += TK_THREADS) {
+                const int64_t i = base + tid;
+                const unsigned long long v = i < nv ? get((int)i) : 0ull;
+                warp_append(v != 0ull && v >= thr, v, sel, &s_nsel, TK_MAX);
+            }
+        }
     }
+    __syncthreads();
     // bitonic sort (descending) of the ke winners, padded with zeros to a power of two
     int n2 = 1;
     while (n2 < ke) n2 <<= 1;

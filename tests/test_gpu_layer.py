@@ -78,7 +78,7 @@ def test_prep_rows_into_the_caches(C):
     tol = 2e-6 * np.abs(ref).max(1, keepdims=True)
     bad = (vg != vr) & (np.abs(vg - ref) > np.abs(vr - ref) + 2 * tol)
     assert not bad.any(), np.argwhere(bad)[:4]
-    assert (vg != vr).mean() < 1e-3
+    assert (f8 != f8r).mean() < 1e-3 and (rb != rbr).mean() < 1e-3   # codes differ only at boundaries
     # index keys: RMSNorm + RoPE + Hadamard -> FP4
     xi = O.bf16_value(O.bf16_bits(g.standard_normal((n, 128)).astype(np.float32))).astype(np.float32)
     gi = np.ones(128, np.float32)
