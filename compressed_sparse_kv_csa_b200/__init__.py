@@ -29,7 +29,7 @@ CSA_BF16 = 1
 CSA_FP4 = 2
 
 EXPORTED = ("csa_compress", "hca_compress", "csa_quantize_kv", "csa_quantize_fp4", "csa_prep_rows",
-            "csa_window_append", "csa_compress_append", "indexer_topk_paged", "hybrid_attn_decode_paged",
+            "csa_window_append", "csa_compress_append", "csa_topk_merge", "indexer_topk_paged", "hybrid_attn_decode_paged",
             "indexer_topk_workspace_size", "indexer_topk", "hybrid_attn_prefill",
             "hybrid_attn_decode_workspace_size", "hybrid_attn_decode", "csa_device_error",
             "csa_status_string", "csa_abi_version", "csa_last_path", "csa_set_wait_limit_ns")
@@ -67,6 +67,7 @@ def _load():
                                ctypes.c_int),
         "hybrid_attn_decode_paged": ([vp, P_kv, vp, i32, i32, vp, P_kv, vp, vp, i32, vp, f32, i32, i32, i32, i32, i32,
                                       i64, vp, vp, vp, sz, vp], ctypes.c_int),
+        "csa_topk_merge": ([vp, vp, vp, i64, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "csa_window_append": ([vp, i32, i64, i32, vp, i32, P_kv, vp], ctypes.c_int),
         "csa_compress_append": ([i32, i64, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, P_kv, P_f4, vp, i32,
                                  i32, vp, vp], ctypes.c_int),
@@ -228,6 +229,17 @@ def csa_quantize_fp4(x, out: Fp4Rows, stream=None):
     _check("csa_quantize_fp4", _lib.csa_quantize_fp4(_ptr(x), _dtype_code(x), n, d, ctypes.byref(out._c()),
                                                      _stream(stream)))
     return out
+
+
+def csa_topk_merge(scores, idx, k: int, bases=None, idx_out=None, score_out=None, stream=None):
+    """Exact top-k of candidate lists stored list-major: scores / idx [n_lists, Nq, list_len]
+    (idx -1 = none), list l's indices offset by bases[l] (int64 device tensor or None)."""
+    n_lists, Nq, list_len = scores.shape
+    if idx_out is None:
+        idx_out = torch.empty((Nq, k), dtype=torch.int32, device=scores.device)
+    _check("csa_topk_merge", _lib.csa_topk_merge(_ptr(scores), _ptr(idx), _ptr(bases), Nq, n_lists, list_len, int(k),
+                                                 _ptr(idx_out), _ptr(score_out), _stream(stream)))
+    return idx_out
 
 
 def csa_window_append(x, pos, W: int, win: KvRows, stream=None):

@@ -351,6 +351,16 @@ int indexer_topk_impl(const void *q, const float *w, const void *keys, int32_t f
 
 extern "C" {
 
+int csa_topk_merge(const float *scores, const int32_t *idx, const int64_t *bases, int64_t Nq, int32_t n_lists,
+                   int32_t list_len, int32_t k, int32_t *idx_out, float *score_out, void *stream)
+{
+    if (!scores || !idx || !idx_out || Nq < 0 || n_lists < 1 || list_len < 1) return CSA_ERR_INVALID_ARG;
+    if (k < 1 || k > 2048 || (int64_t)n_lists * list_len > 16384) return CSA_ERR_UNSUPPORTED;
+    if (Nq == 0) return CSA_OK;
+    return status_of(launch_topk_merge_lists(scores, idx, bases, Nq, n_lists, list_len, k, idx_out, score_out,
+                                             S(stream)));
+}
+
 int indexer_topk_paged(const void *q, const float *w, const void *keys, const int64_t *q_pos, int64_t Nq,
                        int32_t H_I, int32_t d_I, int32_t m, int32_t k, int64_t max_nvis, const int32_t *pages,
                        int32_t max_pages, int32_t page_rows, int32_t *idx_out, float *score_out, void *ws,

@@ -228,6 +228,9 @@ int indexer_topk_impl(const void *q, const float *w, const void *keys, int32_t f
                       void *(*scratch)(cudaError_t *), void *stream, const int32_t *pages = nullptr,
                       int32_t max_pages = 0, int32_t page_rows = 0);
 cudaError_t launch_topk(const IndexerArgs &a, cudaStream_t st);
+cudaError_t launch_topk_merge_lists(const float *scores, const int32_t *idx, const int64_t *bases, int64_t Nq,
+                                    int n_lists, int list_len, int k, int32_t *idx_out, float *score_out,
+                                    cudaStream_t st);
 
 struct PrefillArgs {
     const void *q, *x_win, *kv_comp;

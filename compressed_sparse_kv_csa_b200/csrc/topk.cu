@@ -230,3 +230,103 @@ cudaError_t launch_topk(const IndexerArgs &a, cudaStream_t st)
 }
 
 } // namespace csa
+
+// ------------------------------------------------------------------------------------------
+// merge of candidate lists (the last step of a top-k whose keys were scored in shards)
+// ------------------------------------------------------------------------------------------
+namespace csa {
+
+namespace {
+
+constexpr int TM_THREADS = 512;
+
+// One CTA per query: the exact top-k of its n_lists x list_len (score, index) candidates, stored
+// list-major ([n_lists, Nq, list_len]); list l's indices are offset by bases[l]; index < 0 is
+// ignored.  Ordered by score descending then index ascending.  Candidate keys are staged in
+// shared memory as 64-bit (score key << 32 | ~index) keys, unique when the indices are.
+__global__ void __launch_bounds__(TM_THREADS) topk_merge_lists_kernel(const float *scores, const int32_t *idx,
+                                                                     const int64_t *bases, int64_t Nq, int n_lists,
+                                                                     int list_len, int k, int32_t *idx_out,
+                                                                     float *score_out)
+{
+    const int n_cand = n_lists * list_len;
+    extern __shared__ unsigned long long mk[];
+    __shared__ SelectSmem<uint32_t> msel;
+    __shared__ int s_n, s_w;
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        s_n = 0;
+        s_w = 0;
+    }
+    __syncthreads();
+    for (int j0 = 0; j0 < n_cand; j0 += TM_THREADS) {
+        const int j = j0 + tid;
+        const int l = j / list_len;
+        const int64_t at = ((int64_t)l * Nq + r) * list_len + (j - l * list_len);
+        const int32_t id = j < n_cand ? idx[at] : -1;
+        const bool in = id >= 0;
+        const unsigned long long v = in ? key64(float_key(scores[at]), (int64_t)id + (bases ? bases[l] : 0)) : 0ull;
+        warp_append(in, v, mk, &s_n, n_cand);
+    }
+    __syncthreads();
+    const int n = s_n;
+    const int ke = n < k ? n : k;
+    unsigned long long *sel = mk + n_cand;
+    const unsigned long long thr = n > k ? block_kth64<TM_THREADS>(n, k, [&](int i) { return mk[i]; }, &msel) : 0ull;
+    for (int i = tid; i < n; i += TM_THREADS) {
+        const unsigned long long v = mk[i];
+        if (v >= thr) {
+            const int p = atomicAdd(&s_w, 1);
+            if (p < ke) sel[p] = v;
+        }
+    }
+    __syncthreads();
+    int n2 = 1;
+    while (n2 < ke) n2 <<= 1;
+    for (int i = ke + tid; i < n2; i += TM_THREADS) sel[i] = 0ull;
+    __syncthreads();
+    for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < n2; i += TM_THREADS) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool desc = (i & size) == 0;
+                    const unsigned long long x = sel[i], y = sel[j];
+                    if (desc ? (x < y) : (x > y)) { sel[i] = y; sel[j] = x; }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int j = tid; j < k; j += TM_THREADS) {
+        int32_t id = -1;
+        float sc = -INFINITY;
+        if (j < ke) {
+            const unsigned long long v = sel[j];
+            id = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffu));
+            sc = key_float((uint32_t)(v >> 32));
+        }
+        idx_out[r * k + j] = id;
+        if (score_out) score_out[r * k + j] = sc;
+    }
+}
+
+} // namespace
+
+cudaError_t launch_topk_merge_lists(const float *scores, const int32_t *idx, const int64_t *bases, int64_t Nq,
+                                    int n_lists, int list_len, int k, int32_t *idx_out, float *score_out,
+                                    cudaStream_t st)
+{
+    if (Nq == 0) return cudaSuccess;
+    int n2 = 1;
+    while (n2 < k) n2 <<= 1;
+    const size_t smem = ((size_t)n_lists * list_len + (size_t)n2) * 8;
+    cudaError_t e = cudaFuncSetAttribute(topk_merge_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_merge_lists_kernel<<<(unsigned)Nq, TM_THREADS, smem, st>>>(scores, idx, bases, Nq, n_lists, list_len, k,
+                                                                    idx_out, score_out);
+    return cudaGetLastError();
+}
+
+} // namespace csa

@@ -264,6 +264,23 @@ int indexer_topk_paged(const void *q, const float *w, const void *keys, const in
                        size_t ws_bytes, void *stream);
 
 /*
+ * csa_topk_merge -- the exact top-k of candidate lists: the last step of an indexer top-k whose
+ * keys were scored in shards (one sequence's entries split over several GPUs, each GPU returning
+ * its own k best with indexer_topk(score_out), gathered to every GPU).  The lists are stored
+ * list-major: scores [n_lists, Nq, list_len] fp32 and idx [n_lists, Nq, list_len] int32, list
+ * l's indices offset by bases[l] (int64, or NULL for 0); entries with idx < 0 are ignored.  Per
+ * query r, idx_out [Nq, k] gets the k_eff = min(k, valid candidates) indices with the largest
+ * scores, ordered by score descending, equal scores by lower index, then -1; score_out [Nq, k] (or
+ * NULL) their scores, -inf in padded slots.  The indices of one query must be distinct.  Since
+ * every list holds its shard's k best, the merge is the top-k of the whole sequence ([notes] Sec.
+ * 2.3 Indexer listing; the pages do not shard the indexer: this is the split of one long sequence
+ * across GPUs).  Errors: CSA_ERR_INVALID_ARG for a null array, Nq < 0, n_lists < 1 or
+ * list_len < 1; CSA_ERR_UNSUPPORTED for k outside [1, 2048] or n_lists * list_len > 16384.
+ */
+int csa_topk_merge(const float *scores, const int32_t *idx, const int64_t *bases, int64_t Nq, int32_t n_lists,
+                   int32_t list_len, int32_t k, int32_t *idx_out, float *score_out, void *stream);
+
+/*
  * indexer_topk_static -- indexer_topk for callers that cannot allocate device memory (for
  * example runtimes that reserve the device memory for their own pools up front and give plugins
  * no allocator).  The pages have no counterpart: this is a library convenience.

@@ -105,3 +105,98 @@ def test_bench_main_exits_nonzero_on_mismatch():
     out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "4", "--impl", "reference"],
                          capture_output=True, text=True, timeout=120, cwd=root, env=env)
     assert out.returncode == 2 and "--gpus 4 but WORLD_SIZE=1" in out.stderr
+
+
+# ---------------------------------------------------------------------------------------------
+# sequence-sharded indexer top-k: the exchange and merge of the shards' lists over two ranks
+# ---------------------------------------------------------------------------------------------
+
+def _oracle_shard(q, w, keys_local, m, k, q_pos, base, count, workspace=None):
+    """Stand-in for the GPU shard step on CPU: the oracle's top-k of the slice, positions shifted
+    by the product's own local_positions."""
+    import oracle as O
+    from compressed_sparse_kv_csa_b200 import sharded as SH
+    lp = SH.local_positions(q_pos, m, base).numpy()
+    nv = np.clip((lp + 1) // m, 0, count)
+    idx = np.full((len(lp), k), -1, np.int32)
+    sc = np.full((len(lp), k), -np.inf, np.float64)
+    if count > 0:
+        S = O.indexer_scores(q.numpy(), w.numpy(), keys_local.numpy(), nv)
+        top = O.topk(S, nv, k)
+        idx[:] = top
+        for r in range(len(lp)):
+            for j in range(k):
+                if top[r, j] >= 0:
+                    sc[r, j] = S[r, top[r, j]]
+    return torch.from_numpy(sc), torch.from_numpy(idx)
+
+
+def _oracle_merge(sc_all, idx_all, bases, k):
+    """Stand-in for the GPU merge on CPU: a full sort of the gathered candidates."""
+    G, Nq, kk = sc_all.shape
+    out = np.full((Nq, k), -1, np.int32)
+    for r in range(Nq):
+        cand = [(-float(sc_all[g, r, j]), int(idx_all[g, r, j]) + int(bases[g])) for g in range(G) for j in range(kk)
+                if int(idx_all[g, r, j]) >= 0]
+        cand.sort()
+        out[r, :min(k, len(cand))] = [c[1] for c in cand[:k]]
+    return torch.from_numpy(out)
+
+
+def _sharded_worker(rank: int, world: int, port: int, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from compressed_sparse_kv_csa_b200 import sharded as SH
+        g = np.random.default_rng(50)
+        n, H, d, m, k = 900, 4, 32, 4, 40
+        K = g.standard_normal((n, d))
+        Q = g.standard_normal((5, H, d))
+        W = g.random((5, H))
+        pos = np.array([3599, 2000, 1500, 7, 4 * 460], np.int64)   # N_vis 900, 500, 375, 2, 460
+        base, count = SH.shard_bounds(n, world, rank)
+        out = SH.indexer_topk_sharded(torch.from_numpy(Q), torch.from_numpy(W), torch.from_numpy(K[base:base + count]),
+                                      m, k, torch.from_numpy(pos), n, shard_fn=_oracle_shard, merge_fn=_oracle_merge)
+        dist.barrier()
+        q.put((rank, base, count, out.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_indexer_exchange_and_merge_equal_the_whole_sequence():
+    """Two gloo ranks each hold half of a sequence's index keys; the shards' lists, exchanged by
+    all_gather and merged, give exactly the top-k of the whole sequence on both ranks (queries
+    whose visible entries end in the first shard, straddle both, or see only a few)."""
+    import oracle as O
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=120) for _ in range(2)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (_, b0, c0, out0), (_, b1, c1, out1) = res
+    assert (b0, c0, b1, c1) == (0, 450, 450, 450)
+    g = np.random.default_rng(50)
+    n, H, d, m, k = 900, 4, 32, 4, 40
+    K = g.standard_normal((n, d))
+    Q = g.standard_normal((5, H, d))
+    W = g.random((5, H))
+    pos = np.array([3599, 2000, 1500, 7, 4 * 460], np.int64)
+    ref, _ = O.indexer_topk(Q, W, K, pos, m, k)
+    np.testing.assert_array_equal(out0, ref)
+    np.testing.assert_array_equal(out1, ref)
+
+
+def test_shard_bounds_cover_every_entry_once():
+    from compressed_sparse_kv_csa_b200 import sharded as SH
+    for n, world in [(262144, 8), (1000, 3), (5, 8), (0, 2)]:
+        seen = []
+        for r in range(world):
+            base, count = SH.shard_bounds(n, world, r)
+            seen += list(range(base, base + count))
+        assert seen == list(range(n))
