@@ -475,6 +475,90 @@ class CsaDecode1M:
         self.h_out.copy_(self.o, non_blocking=True)
 
 
+class CsaPrefillFp4(CsaPrefill):
+    """The CSA layer prefill with its indexer in FP4 ([notes] Sec. 2.3 Indexer listing: rotary
+    embedding, Hadamard rotation and FP4 quantisation of the index queries; the indexer's own
+    compressor does the same to its keys, after the entries' RMSNorm).  One step = the two
+    compressions, csa_prep_rows of the index keys (RMSNorm, RoPE at the block's first token,
+    Hadamard, FP4) and of the index queries (RoPE, Hadamard, FP4), the FP4 indexer top-k and the
+    attention."""
+
+    def __init__(self, w, rank, torch, C, device):
+        super().__init__(w, rank, torch, C, device)
+        T, m, Hi, di = w.T, w.m, w.H_I, w.d_I
+        n = T // m
+        self.keys4 = C.Fp4Rows.empty(n, di, device)
+        self.q4 = C.Fp4Rows.empty(T * Hi, di, device)
+        self.gI = torch.ones(di, dtype=torch.float32, device=device)
+        self.kpos = torch.arange(n, dtype=torch.int64, device=device) * m
+        self.qpos = torch.arange(T, dtype=torch.int64, device=device).repeat_interleave(Hi)
+        self.ws = torch.empty((C.indexer_topk_workspace_size(T, n, w.k),), dtype=torch.uint8, device=device)
+        self.launches_per_step = 7  # compress x2, prep x2, FP4 scan, merge, attention
+        # FP4 block-scaled MMAs: the fp4 peak is the measured bf16 peak x 4 (nominal ratio)
+        self.kernels = [("indexer_topk", "tensor_fp4", self.flops), ("csa_prep_rows", "hbm",
+                        float(n * di * 2 + n * 68 + T * Hi * di * 2 + T * Hi * 68)),
+                        ("hybrid_attn_prefill", "tensor", self.flops_attn)]
+
+    def step(self, sp=None):
+        C, w = self.C, self.w
+        with span(sp, "csa_compress"):
+            C.csa_compress(*self.kv_in, self.B, w.m, out=self.kvc)
+            C.csa_compress(*self.ki_in, self.BI, w.m, out=self.keys)
+        with span(sp, "csa_prep_rows"):
+            C.csa_prep_rows(self.keys, g=self.gI, eps=1e-6, rd=64, pos=self.kpos, hadamard=True, out_fp4=self.keys4)
+            C.csa_prep_rows(self.qI.view(-1, w.d_I), rd=64, pos=self.qpos, hadamard=True, out_fp4=self.q4)
+        with span(sp, "indexer_topk"):
+            C.indexer_topk(self.q4, self.wI, self.keys4, w.m, w.k, max_nvis=w.T // w.m, idx_out=self.idx,
+                           workspace=self.ws)
+        with span(sp, "hybrid_attn_prefill"):
+            C.hybrid_attn_prefill(self.q, self.X, self.kvc, self.sink, 1.0, w.m, w.W, idx=self.idx, o=self.o)
+
+
+class CsaDecodeMtp(CsaDecode1M):
+    """Shared-prefix multi-token decode: 8 sequences at 1M context (262,144 compressed entries
+    each, FP8/BF16 rows, FP4 index keys), each with G = 8 consecutive new tokens (positions
+    1,048,569 .. 1,048,576) against its own prefix; every token has its own index query, top-k
+    and window of the last 128 tokens.  One step = indexer_topk (64 queries, 8 per key array) +
+    hybrid_attn_decode (64 queries)."""
+    G = 8
+
+    def __init__(self, w, rank, torch, C, device):
+        super().__init__(w, rank, torch, C, device)   # 8 sequences: caches, keys
+        G, Bn, H, c, Hi, di, W = self.G, w.B, w.H, w.c, w.H_I, w.d_I, w.W
+        seqs = rank_sequences(Bn, rank)
+        nq = Bn * G
+        t0 = w.T - G + 1
+        self.pos = (torch.arange(G, dtype=torch.int64, device=device) + t0).repeat(Bn)
+        self.key_off = torch.arange(Bn, dtype=torch.int64, device=device).repeat_interleave(G) * self.nv
+        wins = []
+        for b in range(Bn):
+            raw = WL.draw(w, "WIN", 0, W + G - 1, seq=seqs[b])     # the sequence's last W + G - 1 raw rows
+            wins += [raw[j:j + W] for j in range(G)]                 # token j's window: rows j .. j+W-1
+        self.win = C.KvRows.empty(nq * W, c, w.rope, device)
+        C.csa_quantize_kv(torch.from_numpy(np.concatenate(wins)).to(device), self.win)
+        self.win_len = torch.full((nq,), W, dtype=torch.int32, device=device)
+        self.q = torch.from_numpy(np.concatenate([WL.draw(w, "q", 0, G, seq=seqs[b]).reshape(G, H, c)
+                                                  for b in range(Bn)])).to(torch.bfloat16).to(device)
+        qx = torch.from_numpy(np.concatenate([WL.draw(w, "qI", 0, G, seq=seqs[b]).reshape(G * Hi, di)
+                                              for b in range(Bn)])).to(device)
+        self.qI = C.Fp4Rows.empty(nq * Hi, di, device)
+        C.csa_quantize_fp4(qx, self.qI)
+        self.wI = torch.from_numpy(np.concatenate([WL.draw(w, "w", 0, G, seq=seqs[b]) for b in range(Bn)])).to(device)
+        self.idx = torch.empty((nq, w.k), dtype=torch.int32, device=device)
+        self.ws = torch.empty((C.indexer_topk_workspace_size(nq, self.nv, w.k),), dtype=torch.uint8, device=device)
+        self.wsd = torch.empty((C.hybrid_attn_decode_workspace_size(nq, H, c, w.k, W, self.nv, True),),
+                               dtype=torch.uint8, device=device)
+        self.o = torch.empty_like(self.q)
+        torch.cuda.synchronize()
+        row = c - w.rope + 2 * w.rope + 4
+        self.bytes = float(Bn * self.nv * (di // 2 + di // 32))      # each sequence's keys once
+        self.bytes_attn = float(nq * (w.k + W) * row + 2 * nq * H * c * 2)
+        self.bytes_step = self.bytes + self.bytes_attn
+        self.tokens = nq
+        self.kernels = [("indexer_topk", "hbm", self.bytes), ("hybrid_attn_decode", "hbm", self.bytes_attn)]
+        self.step_work = ("hbm", self.bytes_step)
+
+
 class _Layer:
     pass
 
@@ -594,6 +678,7 @@ class MixedDecode:
 
 
 WORKLOADS = {"hca_prefill_32k": HcaPrefill, "csa_prefill_64k": CsaPrefill, "csa_decode_1m": CsaDecode1M,
+             "csa_prefill_64k_fp4": CsaPrefillFp4, "csa_decode_1m_mtp": CsaDecodeMtp,
              "mixed_decode_64": MixedDecode}
 
 
@@ -847,7 +932,8 @@ def oracle_repeat(job, target_s: float = 10.0, max_reps: int = 20):
 
 # ---------------------------------------------------------------------------------------------
 
-DEFAULT_WORKLOADS = ("hca_prefill_32k", "csa_prefill_64k", "csa_decode_1m", "mixed_decode_64")
+DEFAULT_WORKLOADS = ("hca_prefill_32k", "csa_prefill_64k", "csa_decode_1m", "mixed_decode_64", "csa_prefill_64k_fp4",
+                     "csa_decode_1m_mtp")
 
 
 def check_world(gpus: int, world: int):
@@ -907,6 +993,11 @@ def roofline(bound, work, ms, pk, src, kernel, traffic=None):
                 "frac": ach / pk["hbm_gbs"], "peak_source": f"{src} HBM copy", "traffic": traffic,
                 "bytes_per_launch": work, "launch_ms": ms}
     ach = work / (ms * 1e-3) / 1e12
+    if bound == "tensor_fp4":  # block-scaled FP4 MMAs: the measured bf16 peak x 4 (nominal fp4 / bf16)
+        peak = 4.0 * pk["bf16_tflops"]
+        return {"bound": "tensor", "kernel": kernel, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "peak_source": f"{src} dense bf16 burst x 4 (nominal FP4 ratio)",
+                "traffic": traffic, "flops_per_launch": work, "launch_ms": ms}
     return {"bound": "tensor", "kernel": kernel, "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
             "frac": ach / pk["bf16_tflops"], "peak_source": f"{src} dense bf16 burst", "traffic": traffic,
             "flops_per_launch": work, "launch_ms": ms}
@@ -918,6 +1009,9 @@ def workload_config(name, w, job, world):
     if w.kind == "csa_decode":
         cfg.update({"B": w.B, "n_comp_per_seq": (w.T + 1) // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
                     "l2": "FP4 key scan (143 MB) and KV cache (1.2 GB) larger than L2"})
+        if w.extra.get("shared_prefix"):
+            cfg.update({"tokens_per_sequence": job.G, "queries": w.B * job.G,
+                        "positions": f"{w.T - job.G + 1} .. {w.T}"})
     elif w.kind == "mixed_decode":
         cfg = {"workload": name, "B": w.B, "layers": list(w.extra["layers"]), "c": w.c,
                "rope_dims": w.rope, "H": w.H, "W": w.W, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
@@ -932,6 +1026,9 @@ def workload_config(name, w, job, world):
     elif w.kind == "csa_prefill":
         cfg.update({"n_comp": w.T // w.m, "k": w.k, "H_I": w.H_I, "d_I": w.d_I,
                     "l2": "inputs larger than L2 (q alone is 4.3 GB)"})
+        if w.extra.get("fp4_indexer"):
+            cfg["indexer"] = ("FP4 E2M1 + E8M0 (keys: RMSNorm, RoPE at the block's first token, Hadamard; "
+                              "queries: RoPE, Hadamard), block-scaled tcgen05")
     else:
         cfg.update({"n_comp": w.T // w.m, "l2": f"inputs larger than L2 (q alone is {w.T * w.H * w.c * 2 / 1e9:.1f} GB)"})
     return cfg

@@ -10,7 +10,7 @@
 // packed two per byte, one E8M0 scale per 32 elements), so the scan feeds them to tcgen05
 // kind::mxf4 MMAs as they are stored: no conversion.
 //
-// Kernel 1 (grid = key chunks x queries, at most one CTA per SM): each CTA streams its chunk of
+// Kernel 1 (one CTA per (query, key chunk)): each CTA streams its chunk of
 // up to 16,384 keys in 128-key tiles through an 8-stage ring:
 //   * producer warp: one lane issues the TMA load of the tile's codes (128 rows x 64 bytes,
 //     64-byte swizzle, the MMA's K-major layout); the 32 lanes copy the tile's scale words
@@ -176,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     uint8_t *sp = smem_raw + (base - raw);
     auto bar = [&](int b) { return base + OFF_BAR + 8u * (uint32_t)b; };
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t r = blockIdx.y;
-    const int slot = blockIdx.x;
+    const int64_t r = (int64_t)blockIdx.x / co.n_slots; // query
+    const int slot = (int)((int64_t)blockIdx.x % co.n_slots);
     const int64_t nv = dec_nvis(a, r);
     const int chunk = query_chunk(nv, co.n_slots);
     const int keep = query_keep(nv, chunk, a.k, co.lcap);
@@ -557,8 +557,16 @@ bool scan_plan(int64_t Nq, int64_t max_nvis, int k, int sms, Plan *p)
     if (p->slots < 1) p->slots = 1;
     int n2 = 1;
     while (n2 < k) n2 <<= 1;
+    // a list needs room for its keep (largest for the query with the fewest chunks: at most k)
+    // plus what one radix digit keeps above it; twice the keep is ample
+    const int keep_max = query_keep(1, kKT, k, 1 << 30) > query_keep(max_nvis, query_chunk(max_nvis, p->slots), k, 1 << 30)
+                             ? query_keep(1, kKT, k, 1 << 30)
+                             : query_keep(max_nvis, query_chunk(max_nvis, p->slots), k, 1 << 30);
+    int64_t lcap = 2 * (int64_t)keep_max;
     const int64_t room = (kMergeSmem - (int64_t)n2 * 8) / ((int64_t)p->slots * 8);
-    p->lcap = (int)(room < kEpiThreads * kR ? room : kEpiThreads * kR);
+    if (lcap > room) lcap = room;
+    if (lcap > kEpiThreads * kR) lcap = kEpiThreads * kR;
+    p->lcap = (int)lcap;
     return p->slots <= kMaxSlots && p->lcap >= query_keep(max_nvis, query_chunk(max_nvis, p->slots), k, 1 << 30);
 }
 
@@ -579,22 +587,19 @@ size_t decode_indexer_need(int64_t Nq, int64_t max_nvis, int k)
     return lists_bytes(Nq, p) + (size_t)Nq * ld * 4 + 256;
 }
 
-// A bound of decode_indexer_need on any device: the merge keeps every list in kMergeSmem bytes,
-// so the lists of one query never exceed that.
+// Workspace of the decode path on the current device (the chunking follows its SM count).
 size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k)
 {
-    (void)k;
-    const size_t ld = (size_t)((max_nvis + 3) / 4 * 4);
-    return (size_t)Nq * ((size_t)kMergeSmem + (size_t)kMaxSlots * 12 + 256) + (size_t)Nq * ld * 4 + 512;
+    return decode_indexer_need(Nq, max_nvis, k) + 256;
 }
 
 bool decode_indexer_eligible(const IndexerArgs &a)
 {
-    if (a.fmt != CSA_FP4 || a.H != kHI || a.d != kDI || a.Nq <= 0 || a.Nq > 65535 || a.max_nvis <= 0) return false;
+    if (a.fmt != CSA_FP4 || a.H != kHI || a.d != kDI || a.Nq <= 0 || a.Nq > (1 << 24) || a.max_nvis <= 0) return false;
     if (a.pages && (a.page_rows < 8 || a.page_rows > kKT || (a.page_rows & (a.page_rows - 1)))) return false;
     if (a.k > 2048 || a.k4.n >= (1ll << 31) || a.Nq * kHI >= (1ll << 31)) return false;
     Plan p;
-    return scan_plan(a.Nq, a.max_nvis, a.k, device_sms(), &p);
+    return scan_plan(a.Nq, a.max_nvis, a.k, device_sms(), &p) && (int64_t)p.slots * a.Nq < (1ll << 31);
 }
 
 cudaError_t launch_indexer_decode(const IndexerArgs &a0, void *ws, cudaStream_t st)
@@ -621,7 +626,7 @@ cudaError_t launch_indexer_decode(const IndexerArgs &a0, void *ws, cudaStream_t 
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    decode_scan_kernel<<<dim3((unsigned)p.slots, (unsigned)a.Nq), kThreads, SMEM_ALLOC, st>>>(a, maps, co);
+    decode_scan_kernel<<<(unsigned)((int64_t)p.slots * a.Nq), kThreads, SMEM_ALLOC, st>>>(a, maps, co);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int n2 = 1;

@@ -18,6 +18,10 @@ Workloads (one per configuration of the hot path):
                      compressed entries (FP8/BF16 KV rows, FP4 index keys), k=1024, W=128
   mixed_decode_64    64 sequences with log-uniform lengths in [4096, 1,048,576], 4 layers
                      HCA, CSA, HCA, CSA
+  csa_prefill_64k_fp4  the CSA prefill with its indexer in FP4: index keys RMS-normalised,
+                     rotated (RoPE on the last 64 dims, Hadamard) and quantised; queries rotated
+                     and quantised the same way
+  csa_decode_1m_mtp  one sequence, 8 consecutive new tokens against the same 1M-token prefix
 """
 from __future__ import annotations
 
@@ -72,6 +76,14 @@ WORKLOADS = {
                                 rope=64, m=4, H=64, H_I=64, d_I=128, k=512, W=128, q_lora=1024),
     "csa_decode_1m": Workload("csa_decode_1m", 4, "csa_decode", "bf16", T=1048576, c=512,
                               rope=64, m=4, H=64, H_I=64, d_I=128, k=1024, W=128, B=8),
+    # variants of the path (FP4 prefill indexer with the layer's row transforms; shared-prefix
+    # multi-token decode): not configurations of their own, measured beside them
+    "csa_prefill_64k_fp4": Workload("csa_prefill_64k_fp4", 7, "csa_prefill", "bf16", T=65536, c=512,
+                                    rope=64, m=4, H=64, H_I=64, d_I=128, k=512, W=128, q_lora=1024,
+                                    extra={"fp4_indexer": True}),
+    "csa_decode_1m_mtp": Workload("csa_decode_1m_mtp", 6, "csa_decode", "bf16", T=1048576, c=512,
+                                  rope=64, m=4, H=64, H_I=64, d_I=128, k=1024, W=128, B=8,
+                                  extra={"shared_prefix": True}),
     "mixed_decode_64": Workload("mixed_decode_64", 5, "mixed_decode", "bf16", c=512, rope=64,
                                 H=64, H_I=64, d_I=128, k=1024, W=128, B=64,
                                 extra={"layers": ("hca", "csa", "hca", "csa"), "m_csa": 4,

@@ -235,7 +235,8 @@ int csa_prep_rows(const void *x, int32_t in_dtype, int64_t n, int32_t d, const f
  *   max_nvis host-side upper bound of nv(r) (sizes the score buffer)
  *   idx_out  [Nq, k] int32;  score_out [Nq, k] fp32 scores of the selected entries (or NULL;
  *            -inf in padded slots)
- *   ws       workspace of at least indexer_topk_workspace_size(Nq, max_nvis, k) bytes
+ *   ws       workspace of at least indexer_topk_workspace_size(Nq, max_nvis, k) bytes, queried
+ *            with the device current (the FP4 decode path's chunking follows its SM count)
  * Limits: 1 <= k <= 2048, 1 <= H_I <= 128, d_I a multiple of 32 (FP4) or 8 and <= 512.
  * Errors: CSA_ERR_INVALID_ARG for a null q, w, keys or idx_out, Nq < 0, n_keys < 0, m < 1,
  * max_nvis < 0, an unknown fmt, w (or dense q / keys) not 16-byte aligned, or FP4 rows that do
