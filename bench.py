@@ -1189,7 +1189,7 @@ def main():
         return 2
 
     if args.impl == "reference":
-        return reference_arm(args, WL.WORKLOADS[names[0]], world, rank)
+        return reference_arm(args, names[0], WL.WORKLOADS[names[0]], world, rank)
 
     import torch
     import torch.distributed as dist
@@ -1243,7 +1243,7 @@ def main():
     return 0
 
 
-def reference_arm(args, w, world, rank):
+def reference_arm(args, name, w, world, rank):
     """The fp64 oracle as the reference implementation, on the host cores (rank 0 only)."""
     if rank != 0:
         return
@@ -1270,7 +1270,8 @@ def reference_arm(args, w, world, rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "T": w.T, "c": w.c, "m": w.m, "H": w.H, "W": w.W},
+        "config": {"workload": name, "T": w.T, "c": w.c, "m": w.m, "H": w.H, "W": w.W,
+                   "parallelism": f"replicas x{world}"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
