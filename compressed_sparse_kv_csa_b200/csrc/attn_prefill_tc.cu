@@ -443,19 +443,9 @@ bool encode_rows512(CUtensorMap *m, const void *base, uint64_t rows, uint32_t bo
 
 } // namespace
 
-cudaError_t launch_attn_prefill_pair(const PrefillArgs &a, cudaStream_t st, bool *handled);
-
-cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled, bool *pair)
+cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled)
 {
     *handled = false;
-    *pair = false;
-    if (!a.idx) { // HCA (every visible entry): two tokens per item on a 2-CTA cluster
-        cudaError_t e = launch_attn_prefill_pair(a, st, pair);
-        if (*pair) {
-            *handled = true;
-            return e;
-        }
-    }
     if (a.dtype != CSA_BF16 || a.H != kH || a.c != kC || a.W != kW || a.T <= 0) return cudaSuccess;
     if (a.idx && a.k > 4096) return cudaSuccess;
     if ((uint64_t)a.T * kH >= (1ull << 31)) return cudaSuccess; // TMA row coordinates are int32
@@ -469,12 +459,8 @@ cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *
     if (!encode_rows512(&maps.kv, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, kKT) ||
         !encode_rows512(&maps.kvg, have_kv ? a.kv_comp : a.x_win, have_kv ? (uint64_t)a.n_comp : (uint64_t)a.T, 1))
         return cudaErrorNotSupported;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
+    const int sms = device_sms();
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const int64_t grid = a.T < sms ? a.T : sms;
     attn_prefill_tc_kernel<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(a, maps);
