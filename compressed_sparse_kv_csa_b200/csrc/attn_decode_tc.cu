@@ -19,7 +19,8 @@
 //      running max moves, and O is rescaled in TMEM, only when a tile raises it by more than 8),
 //      writing P (bf16) to shared memory;
 //   4. O (+)= P V (two M=64 x N=256 x K=128 MMAs, V = the same tile read MN-major) in TMEM.
-// The item's (max, sum, unnormalised O) rows go to the workspace for the split-K merge.
+// The item's (max, sum, unnormalised O) rows go to the workspace for the split-K merge; O is staged
+// through shared memory (the free K and P regions) so that the workspace writes are coalesced.
 // Every wait of the tile chain is bounded by a.wait_ns (2 s unless a caller lowers it); a wait that
 // runs out records CSA_DEVERR_TIMEOUT and every warp leaves the loop at the next CTA barrier.  The
 // wind-down is safe because nothing asynchronous but the MMAs writes into this CTA: q and the key
@@ -40,6 +41,8 @@ constexpr int kMmaWarp = 8;
 constexpr uint32_t OFF_Q = 0;        // 8 sub-tiles [64 x 128 B]   64 KB
 constexpr uint32_t OFF_K = 65536;    // 8 sub-tiles [128 x 128 B]  128 KB
 constexpr uint32_t OFF_P = 196608;   // 2 sub-tiles [64 x 128 B]   16 KB
+constexpr int kStage = kC + 4;       // item end: O staged over the K and P regions, [64 x kStage] fp32
+static_assert(OFF_K + 4u * kH * kStage <= OFF_P + 16384u, "O staging fits the K and P regions");
 constexpr uint32_t OFF_VALID = 212992; // 128 flags
 constexpr uint32_t OFF_ROWS = OFF_VALID + 512; // 128 resolved key rows (int64)
 constexpr int kSeqCache = 1024;                  // per-sequence key counts kept in shared memory
@@ -342,25 +345,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
             ok = __syncthreads_and(ok);
             ph ^= 1;
         }
-        if (warp < 4 && ok) { // (max, sum, unnormalised O) -> workspace (lane l: channels 256-511, l+16: 0-255)
+        if (warp < 4 && ok) { // (max, sum) -> workspace; unnormalised O -> shared memory (rows of kStage floats)
             const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
             if (upper) {
                 part[(int64_t)row * (kC + 2)] = (m_run == -INFINITY) ? -INFINITY : m_run * kLn2; // natural-log max
                 part[(int64_t)row * (kC + 2) + 1] = l_run;
             }
-            float *orow = part + (int64_t)row * (kC + 2) + 2 + (upper ? 256 : 0);
+            // lane l holds channels 256-511 of its head, lane l+16 channels 0-255; the row stride of
+            // kStage floats puts the 8 rows of a quarter-warp's 16-byte stores in distinct banks
+            const uint32_t srow = sK + 4u * (uint32_t)(row * kStage + (upper ? 256 : 0));
             for (int c = 0; c < 8; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tw + 32u * c, r);
                 tmem_ld_wait();
-                // a partial row is (max, sum, acc[512]): acc starts 8 bytes into a 2056-byte row, so
-                // 8-byte stores are the widest that are aligned for every row
 #pragma unroll
-                for (int g = 0; g < 16; ++g)
-                    *reinterpret_cast<float2 *>(orow + 32 * c + 2 * g) =
-                        make_float2(__uint_as_float(r[2 * g]), __uint_as_float(r[2 * g + 1]));
+                for (int g = 0; g < 8; ++g)
+                    sts4(srow + 128u * c + 16u * g, make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]));
             }
             tc_fence_before();
+        }
+        __syncthreads();
+        if (ok) { // every thread: coalesced 8-byte stores (the accumulators start 8 bytes into a partial row)
+            const float *stage = reinterpret_cast<const float *>(sp + OFF_K);
+            for (int i = tid; i < kH * (kC / 2); i += kThreads) {
+                const int h = i / (kC / 2), j = i % (kC / 2);
+                *reinterpret_cast<float2 *>(part + (int64_t)h * (kC + 2) + 2 + 2 * j) =
+                    *reinterpret_cast<const float2 *>(stage + h * kStage + 2 * j);
+            }
         }
         // the item's TMEM and shared memory are free once every warp is past this point
         tc_fence_before();

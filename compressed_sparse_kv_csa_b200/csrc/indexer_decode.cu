@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
 // kernel 2: exact top-k of one query from the published lists (and saturated chunks' scores)
 // ------------------------------------------------------------------------------------------
 constexpr int kMergeThreads = 1024;
-constexpr int kMaxSlots = 256;
+constexpr int kMaxSlots = 256; // list offsets: 8 per lane of one warp
 
 __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a, ChunkOut co)
 {
@@ -418,21 +418,38 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a
     const int k = a.k, ns = co.n_slots;
     const int64_t nv = dec_nvis(a, r);
     const int chunk = query_chunk(nv, ns);
-    if (tid == 0) {
-        int o = 0;
-        for (int sl = 0; sl < ns; ++sl) {
-            s_off[sl] = o;
-            o += co.count[r * ns + sl];
+    const int lane = tid & 31, wid = tid >> 5;
+    if (wid == 0) { // list offsets: lane l sums slots 8l .. 8l+7, then a warp scan
+        int c[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int sl = 8 * lane + j;
+            c[j] = sl < ns ? co.count[r * ns + sl] : 0;
+            sum += c[j];
         }
-        s_off[ns] = o;
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int o = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int sl = 8 * lane + j;
+            if (sl < ns) s_off[sl] = o;
+            o += c[j];
+        }
+        if (lane == 31) s_off[ns] = incl;
     }
     for (int sl = tid; sl < ns; sl += kMergeThreads) s_theta[sl] = co.theta[r * ns + sl];
     __syncthreads();
     const int total = s_off[ns];
-    // 1. the published lists
-    for (int e = tid; e < ns * co.lcap; e += kMergeThreads) {
-        const int sl = e / co.lcap, i = e - sl * co.lcap;
-        if (i < s_off[sl + 1] - s_off[sl]) mv[s_off[sl] + i] = co.list[(r * ns + sl) * (int64_t)co.lcap + i];
+    // 1. the published lists, one warp per list
+    for (int sl = wid; sl < ns; sl += kMergeThreads / 32) {
+        const unsigned long long *src = co.list + (r * ns + sl) * (int64_t)co.lcap;
+        const int o = s_off[sl], c = s_off[sl + 1] - o;
+        for (int i = lane; i < c; i += 32) mv[o + i] = src[i];
     }
     __syncthreads();
     // 2. theta = the k-th largest published key (0 when fewer than k are published), then the
@@ -509,19 +526,7 @@ __global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(IndexerArgs a
     while (n2 < ke) n2 <<= 1;
     for (int i = ke + tid; i < n2; i += kMergeThreads) sel[i] = 0ull;
     __syncthreads();
-    for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < n2; i += kMergeThreads) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    const bool desc = (i & size) == 0;
-                    const unsigned long long x = sel[i], y = sel[j];
-                    if (desc ? (x < y) : (x > y)) { sel[i] = y; sel[j] = x; }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    block_sort_desc64<kMergeThreads>(sel, n2);
     for (int j = tid; j < k; j += kMergeThreads) {
         int32_t id = -1;
         float sc = -INFINITY;

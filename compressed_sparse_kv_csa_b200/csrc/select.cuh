@@ -252,4 +252,48 @@ __device__ unsigned long long block_kth64(int n, int k, Get get, SelectSmem<uint
     return ((unsigned long long)thr_hi << 32) | lo;
 }
 
+// Sorts a[0 .. n2) (n2 a power of two, 64-bit keys) into descending order with a bitonic network.
+// The compare-exchange steps whose partners are less than 32 apart run in registers (element i is
+// held by lane i % 32 of a warp, the partner's key comes by shuffle), so a barrier is taken only
+// for the steps with partners 32 or more apart and once per merge size.  All NT threads of the
+// group call it; the caller synchronises before (a[] complete) and may read a[] right after.
+template <int NT, int BAR = 0>
+__device__ void block_sort_desc64(unsigned long long *a, int n2, int ltid = threadIdx.x)
+{
+    static_assert(NT % 32 == 0, "whole warps");
+    auto reg_steps = [&](int size_lo, int size_hi, int first_stride) {
+        // sizes size_lo..size_hi (powers of two), strides < 32, first size starting at first_stride
+        for (int i0 = 0; i0 < n2; i0 += NT) { // uniform trip count: every lane takes part in the shuffles
+            const int i = i0 + ltid;
+            const bool in = i < n2;
+            unsigned long long v = in ? a[i] : 0ull;
+            for (int size = size_lo; size <= size_hi; size <<= 1) {
+                for (int st = (size == size_lo ? first_stride : size >> 1); st > 0; st >>= 1) {
+                    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, st);
+                    const bool keep_max = ((i & st) == 0) == ((i & size) == 0);
+                    v = keep_max ? (w > v ? w : v) : (w < v ? w : v);
+                }
+            }
+            if (in) a[i] = v;
+        }
+        group_sync<NT, BAR>();
+    };
+    if (n2 < 2) return;
+    reg_steps(2, n2 < 32 ? n2 : 32, 1);
+    for (int size = 64; size <= n2; size <<= 1) {
+        for (int st = size >> 1; st >= 32; st >>= 1) {
+            for (int i = ltid; i < n2; i += NT) {
+                const int j = i ^ st;
+                if (j > i) {
+                    const bool desc = (i & size) == 0;
+                    const unsigned long long x = a[i], y = a[j];
+                    if (desc ? (x < y) : (x > y)) { a[i] = y; a[j] = x; }
+                }
+            }
+            group_sync<NT, BAR>();
+        }
+        reg_steps(size, size, 16);
+    }
+}
+
 } // namespace csa

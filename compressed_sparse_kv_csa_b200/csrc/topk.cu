@@ -187,19 +187,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     while (n2 < ke) n2 <<= 1;
     for (int i = ke + tid; i < n2; i += TK_THREADS) sel[i] = 0ull;
     __syncthreads();
-    for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < n2; i += TK_THREADS) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    const bool desc = (i & size) == 0;
-                    const unsigned long long x = sel[i], y = sel[j];
-                    if (desc ? (x < y) : (x > y)) { sel[i] = y; sel[j] = x; }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    block_sort_desc64<TK_THREADS>(sel, n2);
     for (int j = tid; j < k; j += TK_THREADS) {
         int32_t id = -1;
         float sc = -INFINITY;
@@ -286,19 +274,7 @@ __global__ void __launch_bounds__(TM_THREADS) topk_merge_lists_kernel(const floa
     while (n2 < ke) n2 <<= 1;
     for (int i = ke + tid; i < n2; i += TM_THREADS) sel[i] = 0ull;
     __syncthreads();
-    for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < n2; i += TM_THREADS) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    const bool desc = (i & size) == 0;
-                    const unsigned long long x = sel[i], y = sel[j];
-                    if (desc ? (x < y) : (x > y)) { sel[i] = y; sel[j] = x; }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    block_sort_desc64<TM_THREADS>(sel, n2);
     for (int j = tid; j < k; j += TM_THREADS) {
         int32_t id = -1;
         float sc = -INFINITY;
