@@ -8,11 +8,12 @@
 // One CTA of 512 threads per query row; rows of at most TK_STAGE scores are staged in shared
 // memory as order-preserving 32-bit keys.  Every entry has the unique 64-bit key
 // (score key << 32 | ~index), so "the k largest keys" is exactly the wanted set.  Three passes
-// over the row: (1) the range of the score keys; (2) a histogram of the top 11 bits of the keys
-// offset by the minimum and left-aligned on the range (2,048 bins, warp-aggregated atomics), whose
-// suffix sums give the bin b* that holds the k-th key; (3) keys in bins above b* are winners,
+// over the row: (1) the range of the score keys (taken while staging); (2) a histogram of the top
+// 11 bits of the keys offset by the minimum and left-aligned on the range (2,048 bins, shared-memory
+// atomics), whose suffix sums give the bin b* that holds the k-th key; (3) keys in bins above b* are winners,
 // keys in b* are candidates (warp-aggregated appends).  The few candidates are resolved by an
-// exact 64-bit selection, and the k winners are sorted in shared memory (bitonic).
+// exact 64-bit selection, and the k winners are sorted in shared memory (bitonic; the steps
+// between elements less than 32 apart by warp shuffles).
 #include "common.cuh"
 #include "select.cuh"
 
@@ -73,13 +74,19 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     const int k = a.k;
     const int ke = (int)(nv < k ? nv : k);
     const float *S = a.scores + r * a.ld;
+    uint32_t lo = 0xffffffffu, hi = 0; // range of this thread's keys (the staging pass takes it)
     if (STAGED) { // rows are 16-byte aligned and padded to a multiple of 4 scores
         for (int64_t i4 = tid; 4 * i4 < nv; i4 += TK_THREADS) {
             const float4 v = *reinterpret_cast<const float4 *>(S + 4 * i4);
-            skeys[4 * i4 + 0] = float_key(v.x);
-            skeys[4 * i4 + 1] = float_key(v.y);
-            skeys[4 * i4 + 2] = float_key(v.z);
-            skeys[4 * i4 + 3] = float_key(v.w);
+            const uint32_t k4[4] = {float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w)};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                skeys[4 * i4 + u] = k4[u];
+                if (4 * i4 + u < nv) {
+                    lo = k4[u] < lo ? k4[u] : lo;
+                    hi = k4[u] > hi ? k4[u] : hi;
+                }
+            }
         }
     }
     if (tid == 0) {
@@ -93,12 +100,13 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
     if (nv <= k) { // every visible entry is a winner
         for (int64_t i = tid; i < nv; i += TK_THREADS) sel[i] = key64(key(i), i);
     } else {
-        // 1. range of the score keys
-        uint32_t lo = 0xffffffffu, hi = 0;
-        for (int64_t i = tid; i < nv; i += TK_THREADS) {
-            const uint32_t v = key(i);
-            lo = v < lo ? v : lo;
-            hi = v > hi ? v : hi;
+        // 1. range of the score keys (already taken by the staging pass)
+        if (!STAGED) {
+            for (int64_t i = tid; i < nv; i += TK_THREADS) {
+                const uint32_t v = key(i);
+                lo = v < lo ? v : lo;
+                hi = v > hi ? v : hi;
+            }
         }
         lo = warp_min_key(lo);
         hi = warp_max_key(hi);
@@ -115,14 +123,9 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(IndexerArgs a)
         }
         const int lead = (hi == lo) ? 32 : __clz(hi - lo);
         auto bin_of = [&](uint32_t v) -> int { return lead >= 32 ? 0 : (int)(((v - lo) << lead) >> 21); };
-        // 2. histogram of the 11-bit first digit (lanes with the same bin add once)
-        for (int64_t base = 0; base < nv; base += TK_THREADS) {
-            const int64_t i = base + tid;
-            const bool in = i < nv;
-            const int b = in ? bin_of(key(i)) : -1;
-            const unsigned peers = __match_any_sync(0xffffffffu, b);
-            if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[b], __popc(peers));
-        }
+        // 2. histogram of the 11-bit first digit (shared-memory atomics; the range-normalised bins
+        //    spread a warp's keys, so lanes rarely collide)
+        for (int64_t i = tid; i < nv; i += TK_THREADS) atomicAdd(&hist[bin_of(key(i))], 1);
         __syncthreads();
         if (wid == 0) { // suffix scan from the top bin: lane l owns bins 2047-64l .. 1984-64l
             int sum = 0;
