@@ -43,10 +43,10 @@ constexpr uint32_t OFF_K = 65536;    // 8 sub-tiles [128 x 128 B]  128 KB
 constexpr uint32_t OFF_P = 196608;   // 2 sub-tiles [64 x 128 B]   16 KB
 constexpr int kStage = kC + 4;       // item end: O staged over the K and P regions, [64 x kStage] fp32
 static_assert(OFF_K + 4u * kH * kStage <= OFF_P + 16384u, "O staging fits the K and P regions");
-constexpr uint32_t OFF_VALID = 212992; // 128 flags
-constexpr uint32_t OFF_ROWS = OFF_VALID + 512; // 128 resolved key rows (int64)
+constexpr uint32_t OFF_VALID = 212992;          // 2 x 128 flags (this tile, the next)
+constexpr uint32_t OFF_ROWS = OFF_VALID + 1024;  // 2 x 128 resolved key rows (int64)
 constexpr int kSeqCache = 1024;                  // per-sequence key counts kept in shared memory
-constexpr uint32_t OFF_SEQ = OFF_ROWS + 1024;    // n_win [kSeqCache], n_keys [kSeqCache] (int32)
+constexpr uint32_t OFF_SEQ = OFF_ROWS + 2048;    // n_win [kSeqCache], n_keys [kSeqCache] (int32)
 constexpr uint32_t OFF_BAR = OFF_SEQ + 8 * kSeqCache;
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = OFF_TMEM + 64 + 1024;
@@ -143,10 +143,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
     const bool upper = lane < 16;
     const int row = 16 * (warp & 3) + (lane & 15); // head of this softmax lane (warps 0-3)
     const float sl2 = a.scale * kLog2e;
+    int b = 0, n_win = 0;
+    int64_t n_keys = 0;
+    // key j of sequence b: window row, or compressed row | 2^62, or -1 = empty; stored in slot sl
+    auto resolve = [&](int64_t j, int64_t *rw, int *vd, int sl) -> int64_t {
+        int64_t code = -1;
+        if (j < n_keys && j < n_win) {
+            code = (int64_t)b * a.W + j;
+        } else if (j < n_keys) {
+            const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
+            if (s >= 0) { // a selected entry that is missing or not yet visible is skipped and reported
+                int64_t nvb = (a.pos[b] + 1) / a.m;
+                nvb = nvb > a.max_nvis ? a.max_nvis : nvb;
+                const int64_t r = paged_row(a.pages, a.max_pages, a.page_rows, b, s, a.pages ? 0 : a.comp_off[b]);
+                if (s < nvb && r >= 0 && r < a.comp.n) code = r | (1ll << 62);
+                else flag_error(a.err, CSA_DEVERR_INDEX);
+            }
+        }
+        rw[sl] = code;
+        vd[sl] = code >= 0 ? 1 : 0;
+        return code;
+    };
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int b = (int)(item / a.n_chunks), chunk = (int)(item % a.n_chunks);
-        int n_win;
-        int64_t n_keys;
+        b = (int)(item / a.n_chunks); // the sequence and key counts resolve() reads
+        const int chunk = (int)(item % a.n_chunks);
         if (b < kSeqCache) {
             n_win = s_nwin[b];
             n_keys = s_nkeys[b];
@@ -184,26 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
         float m_run = -INFINITY, l_run = 0.f; // online softmax of this lane's row (log2 domain)
         for (int64_t tile = t_beg; tile < t_end && ok; ++tile) {
             const bool first = tile == t_beg;
-            const int64_t j0 = tile * kKT;
-            // ---- resolve the tile's 128 key slots: window row, or compressed row | 2^62, or -1 = empty
-            if (tid < kKT) {
-                const int64_t j = j0 + tid;
-                int64_t code = -1;
-                if (j < n_keys && j < n_win) {
-                    code = (int64_t)b * a.W + j;
-                } else if (j < n_keys) {
-                    const int64_t s = a.idx ? (int64_t)a.idx[(int64_t)b * a.k + (j - n_win)] : (j - n_win);
-                    if (s >= 0) { // a selected entry that is missing or not yet visible is skipped and reported
-                        int64_t nvb = (a.pos[b] + 1) / a.m;
-                        nvb = nvb > a.max_nvis ? a.max_nvis : nvb;
-                        const int64_t r = paged_row(a.pages, a.max_pages, a.page_rows, b, s, a.pages ? 0 : a.comp_off[b]);
-                        if (s < nvb && r >= 0 && r < a.comp.n) code = r | (1ll << 62);
-                        else flag_error(a.err, CSA_DEVERR_INDEX);
-                    }
-                }
-                rows[tid] = code;
-                valid[tid] = code >= 0 ? 1 : 0;
-            }
+            const int buf = (int)((tile - t_beg) & 1);
+            int64_t *rw = rows + kKT * buf;
+            int *vd = valid + kKT * buf;
+            // ---- the item's first tile resolves its 128 key slots here; later tiles were resolved
+            // (and their rows prefetched into L2) while the previous tile was computed
+            if (first && tid < kKT) resolve(tile * kKT + tid, rw, vd, tid);
             __syncthreads();
             // ---- gather the key rows, FP8 part dequantised to bf16 (code x row scale), RoPE part as
             // is; 12 independent loads per thread in flight
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
                     raw[u] = make_uint4(0, 0, 0, 0);
                     sc[u] = 0.f;
                     if (e < kKT * (kC / 8)) {
-                        const int64_t code = rows[e >> 6];
+                        const int64_t code = rw[e >> 6];
                         if (code >= 0) {
                             const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
                             const int64_t rw = code & ((1ll << 62) - 1);
@@ -251,6 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
+            // warps 4-7 have nothing to do until the next gather: resolve the next tile of the item
+            // into the other row buffer and start its rows on their way into L2
+            if (warp >= 4 && warp < 8 && tile + 1 < t_end) {
+                const int sl = tid - 128;
+                const int64_t code = resolve((tile + 1) * kKT + sl, rows + kKT * (buf ^ 1), valid + kKT * (buf ^ 1), sl);
+                if (code >= 0) {
+                    const KvRowsDev &kv = (code >> 62) ? a.comp : a.win;
+                    const int64_t rr = code & ((1ll << 62) - 1);
+                    const uint8_t *f8 = kv.fp8 + rr * cn;
+                    for (int o = 0; o < cn; o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(f8 + o));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(kv.rope + rr * kv.rope_dims));
+                }
+            }
 
             if (warp == kMmaWarp && lane == 0) { // S = Q K^T
 #pragma unroll
@@ -280,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(DecodeArgs 
                         const uint32_t x = __shfl_xor_sync(0xffffffffu, r2[e], 16);
                         const uint32_t y = __shfl_xor_sync(0xffffffffu, r3[e], 16);
                         float s0 = __uint_as_float(upper ? r0[e] : x), s1 = __uint_as_float(upper ? r1[e] : y);
-                        s0 = valid[kb + e] ? s0 * sl2 : -INFINITY;
-                        s1 = valid[kb + 32 + e] ? s1 * sl2 : -INFINITY;
+                        s0 = vd[kb + e] ? s0 * sl2 : -INFINITY;
+                        s1 = vd[kb + 32 + e] ? s1 * sl2 : -INFINITY;
                         sv[e] = s0;
                         sv[32 + e] = s1;
                         mt = fmaxf(mt, fmaxf(s0, s1));
