@@ -48,7 +48,7 @@ using namespace tc;
 
 constexpr int kHI = 64, kDI = 128, kKT = 128, kStages = 8;
 constexpr int kChunk = 16384;                 // most keys per CTA
-constexpr int kR = 16;                        // keys kept per epilogue thread
+constexpr int kR = 8;                         // keys kept per epilogue thread
 constexpr int kMergeSmem = 200 * 1024;        // merge kernel: published lists + winners
 constexpr int kShareMax = 512;                // most of k one chunk is expected to hold
 constexpr int kProdWarp = 0, kEpiWarp0 = 1, kEpiWarps = 8, kMmaWarp = kEpiWarp0 + kEpiWarps;
