@@ -587,11 +587,17 @@ class MixedDecode:
             L.m = w.extra["m_csa"] if L.csa else w.extra["m_hca"]
             nv = (self.lens + 1) // L.m
             L.nv, L.max_nv = nv, int(nv.max())
-            L.off_np = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+            # every sequence's compressed rows start at a multiple of 32 rows (a 128-token page of a
+            # CSA layer), as a paged cache allocator places them
+            seg = (nv + 31) // 32 * 32
+            L.off_np = np.concatenate([[0], np.cumsum(seg)[:-1]]).astype(np.int64)
             L.off = torch.from_numpy(L.off_np).to(device)
-            n = int(nv.sum())
+            n = int(seg.sum())
             L.comp = C.KvRows.empty(n, c, w.rope, device)
             L.keys = C.Fp4Rows.empty(n, di, device) if L.csa else None
+            if L.csa:  # rows past a sequence's entries are never selected, but the scan's tiles read them
+                L.keys.codes.zero_()
+                L.keys.scales.zero_()
             chunk = 65536
             for b in range(Bn):
                 o0 = int(L.off_np[b])

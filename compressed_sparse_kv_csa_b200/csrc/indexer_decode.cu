@@ -85,6 +85,10 @@ enum { M_COUNT = 0, M_ABORT = 1, M_OUT = 2, M_RED = 4 }; // M_RED: 8 x u64 (one 
 
 struct Maps {
     CUtensorMap q, k, kp; // kp: key rows in boxes of one page (paged caches only)
+    // Permuted tiles (see the scan kernel): every 4th key row (kq4: 32 rows a box, kq4p: a page's
+    // share), the scale words as rows of 4 (sq: 32 rows a box, sqp: a page's share)
+    CUtensorMap kq4, kq4p, sq, sqp;
+    int perm; // the permuted maps exist (and, when paged, pages hold >= 32 rows)
 };
 
 __device__ __forceinline__ int64_t dec_nvis(const IndexerArgs &a, int64_t r)
@@ -194,13 +198,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
     }
     const int64_t key0 = (a.key_off ? a.key_off[r] : 0) + c0; // first key row of the chunk
     const int ntiles = (n + kKT - 1) / kKT;
+    // Permuted tiles: MMA row 32j + l holds key 4l + j of the tile, so that the scale words of the
+    // keys on TMEM lane l (keys 4l .. 4l+3 in columns j = 0..3 of the block-scale layout) are 16
+    // contiguous bytes, and a tile's 128 scale words arrive by TMA as they are stored.  The codes
+    // come as four boxes of every 4th row.  Needs the chunk to start at a multiple of 4 rows.
+    const bool perm = maps.perm && (a.pages || (key0 & 3) == 0);
     int *misc = reinterpret_cast<int *>(sp + OFF_MISC);
     unsigned long long *red = reinterpret_cast<unsigned long long *>(sp + OFF_MISC + 4 * M_RED);
 
     if (tid == 0) {
         for (int b = 0; b < NUM_BARS; ++b) {
             uint32_t cnt = 1;
-            if (b >= B_FULL && b < B_FULL + kStages) cnt = 1 + 32; // expect_tx arrive + 32 cp.async arrivals
+            if (b >= B_FULL && b < B_FULL + kStages) cnt = perm ? 1 : 1 + 32; // expect_tx arrive (+ 32 cp.async arrivals)
             if (b >= B_DEMPTY && b < B_DEMPTY + kDBufs) cnt = 4;
             mbar_init(bar(b), cnt);
         }
@@ -235,6 +244,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             const int64_t row0 = key0 + (int64_t)i * kKT;
             const int valid = n - i * kKT < kKT ? n - i * kKT : kKT; // keys of the chunk in this tile
             const int64_t e0 = c0 + (int64_t)i * kKT;                // the tile's first entry
+            if (perm) { // codes and scale words by TMA only
+                if (lane == 0) {
+                    const uint32_t dst = base + OFF_ST + st * kTileCodes, sdst = base + OFF_SCL + st * 512u;
+                    mbar_arrive_expect_tx(bar(B_FULL + st), kTileCodes + 512u);
+                    if (!a.pages) {
+                        const int32_t y0 = (int32_t)(row0 >> 2);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) tma_load_3d(dst + 2048u * j, &maps.kq4, 0, j, y0, bar(B_FULL + st));
+                        tma_load_2d(sdst, &maps.sq, 0, y0, bar(B_FULL + st));
+                    } else { // per page: its rows 4m + j and its scale words; a bad page reads page 0
+                        const int pr4 = a.page_rows >> 2;
+                        for (int u = 0; u * a.page_rows < kKT; ++u) {
+                            const int64_t eu = e0 + (int64_t)u * a.page_rows;
+                            int64_t prow = eu < c0 + n ? paged_row(a.pages, a.max_pages, a.page_rows, r, eu, 0) : 0;
+                            if (prow < 0 || prow >= a.k4.n) prow = 0;
+                            const int32_t y0 = (int32_t)(prow >> 2);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                tma_load_3d(dst + (uint32_t)(32 * j + pr4 * u) * 64u, &maps.kq4p, 0, j, y0, bar(B_FULL + st));
+                            tma_load_2d(sdst + (uint32_t)(pr4 * u) * 16u, &maps.sqp, 0, y0, bar(B_FULL + st));
+                        }
+                    }
+                }
+                continue;
+            }
             for (int j = lane; j < valid; j += 32) {
                 const int64_t row = a.pages ? paged_row(a.pages, a.max_pages, a.page_rows, r, e0 + j, 0) : row0 + j;
                 if (row >= 0 && row < a.k4.n) // a bad page leaves the word unset; the epilogue drops the key
@@ -293,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_scan_kernel(IndexerArgs a,
             for (int h = 0; h < 32; ++h)
                 acc[h & 3] = fmaf(w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), acc[h & 3]);
             const float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            const int kc = i * kKT + 32 * quad + lane;
+            const int kc = i * kKT + (perm ? 4 * lane + quad : 32 * quad + lane); // key of TMEM lane 32 quad + lane
             bool live = kc < n;
             if (live && a.pages) { // a key whose page is missing or out of range is dropped and reported
                 const int64_t row = paged_row(a.pages, a.max_pages, a.page_rows, r, c0 + kc, 0);
@@ -629,6 +663,15 @@ cudaError_t launch_indexer_decode(const IndexerArgs &a0, void *ws, cudaStream_t 
         return cudaErrorInvalidValue;
     if (a.pages && !tma::encode_u8_rows_sw64(&maps.kp, a.k4.codes, key_rows, kDI / 2, (uint32_t)a.page_rows))
         return cudaErrorInvalidValue;
+    // permuted tiles when the key rows come in whole groups of 4 and the arrays are 16-byte aligned
+    // (the encoder checks); otherwise every tile takes the natural order
+    maps.perm = (key_rows % 4 == 0) && (!a.pages || a.page_rows >= 32) &&
+                tma::encode_u8_rows_sw64_stride4(&maps.kq4, a.k4.codes, key_rows, kKT / 4) &&
+                tma::encode_u32_quads(&maps.sq, a.k4.scales, key_rows, kKT / 4) &&
+                (!a.pages || (tma::encode_u8_rows_sw64_stride4(&maps.kq4p, a.k4.codes, key_rows, (uint32_t)a.page_rows / 4) &&
+                              tma::encode_u32_quads(&maps.sqp, a.k4.scales, key_rows, (uint32_t)a.page_rows / 4)))
+                    ? 1
+                    : 0;
     cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     decode_scan_kernel<<<(unsigned)((int64_t)p.slots * a.Nq), kThreads, SMEM_ALLOC, st>>>(a, maps, co);

@@ -109,6 +109,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
                  : "memory");
 }
 
+// 3-D tiled TMA load (no multicast) of the box at (x, y, z); x must be a multiple of 16 bytes /
+// element size.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+                 : "memory");
+}
+
 // TMA gather of 4 rows (y0..y3) x the box width at column x (2-D map with a one-row box) into
 // shared memory as a 4-row block; completes 4 x box bytes of the transaction count of `bar`.
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int32_t x, int32_t y0, int32_t y1,

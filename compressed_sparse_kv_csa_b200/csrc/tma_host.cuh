@@ -54,5 +54,36 @@ inline bool encode_u8_rows_sw64(CUtensorMap *m, const void *base, uint64_t rows,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Every 4th row of a [rows, 64]-byte matrix: the 3-D view {64 bytes, 4 (row mod 4), rows / 4} read
+// in boxes of 64 bytes x 1 x box_rows with the 64-byte swizzle, so that box (0, j, y) holds rows
+// 4y + j, 4(y+1) + j, ...; rows must be a multiple of 4; rows outside read as zeros.
+inline bool encode_u8_rows_sw64_stride4(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+    if (!enc || rows < 4 || rows % 4 || box_rows == 0 || box_rows > 256) return false;
+    const cuuint64_t dims[3] = {64, 4, (cuuint64_t)(rows / 4)};
+    const cuuint64_t strides[2] = {64, 256};
+    const cuuint32_t box[3] = {64, 1, box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A vector of 32-bit words viewed as rows of 4 words ({4, words / 4}), read in boxes of 4 x
+// box_rows without swizzle; words must be a multiple of 4; rows outside read as zeros.
+inline bool encode_u32_quads(CUtensorMap *m, const void *base, uint64_t words, uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+    if (!enc || words < 4 || words % 4 || box_rows == 0 || box_rows > 256) return false;
+    const cuuint64_t dims[2] = {4, (cuuint64_t)(words / 4)};
+    const cuuint64_t strides[1] = {16};
+    const cuuint32_t box[2] = {4, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 } // namespace tma
 } // namespace csa

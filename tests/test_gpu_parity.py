@@ -194,6 +194,48 @@ def test_indexer_topk_fp4_decode_batches(C):
     assert check_topk(idx.cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
 
 
+@pytest.mark.parametrize("shift,extra", [(1, 0), (2, 0), (0, 3)])
+def test_fp4_scan_tile_orders_agree(C, shift, extra):
+    """The FP4 scan takes a tile's keys in two orders: permuted (MMA row 32j + l = key 4l + j, codes
+    and scale words by TMA alone) when a chunk starts at a multiple of 4 rows and the key array
+    holds whole groups of 4 rows, else in natural order (scale words by cp.async).  The same keys in
+    aligned segments, and again moved down by `shift` rows or in an array `extra` rows longer (not
+    a multiple of 4), give the same indices and scores bit for bit, and agree with the oracle."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, H, d, k, m = 4, 64, 128, 512, 4
+    pos = np.array([4 * 20000 - 1, 4 * 9000 + 1, 4 * 700 + 2, 4 * 130 - 1], np.int64)
+    nv = O.n_vis(pos, m)
+    seg = (nv + 3) // 4 * 4 + 4                       # aligned segments (with room for the shift)
+    off = np.concatenate([[0], np.cumsum(seg)[:-1]]).astype(np.int64)
+    n_rows = int(seg.sum())
+    keys = np.zeros((n_rows, d), np.float32)
+    for b in range(Bn):
+        keys[off[b]:off[b] + nv[b]] = WL.draw(w, "KI", 0, int(nv[b]), seq=30 + b)
+    qx = np.stack([WL.draw(w, "qI", 0, 1, seq=30 + b).reshape(H, d) for b in range(Bn)])
+    wt = dev(np.concatenate([WL.draw(w, "w", 0, 1, seq=30 + b) for b in range(Bn)]))
+    q4 = C.Fp4Rows.empty(Bn * H, d, "cuda")
+    C.csa_quantize_fp4(dev(qx.reshape(Bn * H, d)), q4)
+    pos_d = torch.from_numpy(pos).cuda()
+    outs = []
+    for sh, ex in ((0, 0), (shift, extra)):
+        kk = np.zeros((n_rows + ex, d), np.float32)
+        kk[sh:n_rows] = keys[:n_rows - sh]
+        k4 = C.Fp4Rows.empty(n_rows + ex, d, "cuda")
+        C.csa_quantize_fp4(dev(kk), k4)
+        sc = torch.empty((Bn, k), dtype=torch.float32, device="cuda")
+        idx = C.indexer_topk(q4, wt, k4, m, k, max_nvis=int(nv.max()), q_pos=pos_d,
+                             key_off=torch.from_numpy(off + sh).cuda(), score_out=sc)
+        assert C.csa_last_path() == C.CSA_PATH_INDEXER_FP4_TC
+        outs.append((idx, sc))
+    torch.cuda.synchronize()
+    assert C.csa_device_error() == 0
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    Kd = O.dequant_fp4(*O.quant_fp4(keys))
+    Qd = O.dequant_fp4(*O.quant_fp4(qx.reshape(Bn * H, d))).reshape(Bn, H, d)
+    idx_o, S = O.indexer_topk(Qd, host(wt), Kd, pos, m, k, kbase=off)
+    assert check_topk(outs[0][0].cpu().numpy(), idx_o, S, nv, k) >= Bn - 1
+
+
 @pytest.mark.parametrize("Bn,k", [(16, 1024), (12, 2048)])
 def test_fp4_decode_streaming_filter(C, Bn, k):
     """Chunks longer than the scan's candidate buffer (16 or 12 sequences of 40-60k entries), so
