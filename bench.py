@@ -755,17 +755,20 @@ class OracleDecode:
         import oracle as O
         self.w, self.n = w, n_seq
         H, c, Hi, di, W, m = w.H, w.c, w.H_I, w.d_I, w.W, w.m
-        self.t = w.T
+        self.G = 8 if w.extra.get("shared_prefix") else 1   # new tokens per sequence
+        G = self.G
+        self.t = np.arange(w.T - G + 1, w.T + 1, dtype=np.int64)
         self.nv = (w.T + 1) // m
         self.seqs = []
         for b in range(n_seq):
             s = b + w.B * seed_rank
             Kd = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "KI", 0, self.nv, seq=s)))
             KV = O.dequant_kv(*O.quant_kv(WL.draw(w, "KV", 0, self.nv, seq=s)))
-            win = O.dequant_kv(*O.quant_kv(WL.draw(w, "WIN", 0, W, seq=s)))
-            q = WL.draw(w, "q", 0, 1, seq=s).reshape(1, H, c)
-            qI = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "qI", 0, 1, seq=s).reshape(Hi, di))).reshape(1, Hi, di)
-            wt = WL.draw(w, "w", 0, 1, seq=s)
+            raw = WL.draw(w, "WIN", 0, W + G - 1, seq=s)   # token j's window: rows j .. j+W-1
+            win = O.dequant_kv(*O.quant_kv(np.concatenate([raw[j:j + W] for j in range(G)])))
+            q = WL.draw(w, "q", 0, G, seq=s).reshape(G, H, c)
+            qI = O.dequant_fp4(*O.quant_fp4(WL.draw(w, "qI", 0, G, seq=s).reshape(G * Hi, di))).reshape(G, Hi, di)
+            wt = WL.draw(w, "w", 0, G, seq=s)
             self.seqs.append((Kd, KV, win, q, qI, wt))
         self.sink = WL.draw(w, "sink", 0, 1, seq=seed_rank)[0]
 
@@ -774,14 +777,16 @@ class OracleDecode:
         import oracle as O
         w = self.w
         t0 = time.perf_counter()
+        G = self.G
         for Kd, KV, win, q, qI, wt in self.seqs:
-            idx, _ = O.indexer_topk(qI, wt, Kd, np.array([self.t]), w.m, w.k)
-            O.hybrid_attn_decode(q, KV, [0], [self.t], win, [w.W], self.sink, 1.0, w.m, w.W, idx=idx)
+            idx, _ = O.indexer_topk(qI, wt, Kd, self.t, w.m, w.k)
+            O.hybrid_attn_decode(q, KV, [0] * G, self.t, win, [w.W] * G, self.sink, 1.0, w.m, w.W, idx=idx)
         secs = time.perf_counter() - t0
-        return self.n / secs, secs
+        return self.n * G / secs, secs
 
     def describe(self):
-        return (f"{self.n} of the {self.w.B} sequences: FP4 indexer over {self.nv} entries, top-{self.w.k}, "
+        toks = f", {self.G} new tokens each" if self.G > 1 else ""
+        return (f"{self.n} of the {self.w.B} sequences{toks}: FP4 indexer over {self.nv} entries, top-{self.w.k}, "
                 f"hybrid attention over the selected rows + window {self.w.W}")
 
 
@@ -895,9 +900,17 @@ class OracleCsa:
         t0 = time.perf_counter()
         KV = O.csa_compress(*self.kv_in, self.B, w.m)
         KI = O.csa_compress(*self.ki_in, self.BI, w.m)
+        fp4 = bool(w.extra.get("fp4_indexer"))
+        if fp4:  # index keys: RMSNorm, RoPE at the block's first token, Hadamard, FP4
+            KI = O.rope(O.rmsnorm(KI, np.ones(KI.shape[1]), 1e-6), np.arange(KI.shape[0]) * w.m, 64)
+            KI = O.dequant_fp4(*O.quant_fp4(O.hadamard(KI)))
         t_comp = time.perf_counter() - t0
         t1 = time.perf_counter()
         for rows, q, qI, wI in zip(self.rows, self.q, self.qI, self.wI):
+            if fp4:  # index queries: RoPE at the token's position, Hadamard, FP4
+                n_r, hi, di = qI.shape
+                x = O.rope(qI.reshape(n_r * hi, di), np.repeat(rows, hi), 64)
+                qI = O.dequant_fp4(*O.quant_fp4(O.hadamard(x))).reshape(n_r, hi, di)
             idx, _ = O.indexer_topk(qI, wI, KI, rows, w.m, w.k)
             by_pos = {int(t): idx[i] for i, t in enumerate(rows)}   # the oracle looks rows up by position
             O.hybrid_attn_prefill(q, self.X, KV, self.sink, 1.0, w.m, w.W, idx=by_pos, rows=rows)
@@ -906,7 +919,8 @@ class OracleCsa:
         return 1.0 / per_token, t_comp + t_tok, t_comp, t_tok
 
     def describe(self):
-        return (f"full csa_compress of the KV entries and the index keys (T={self.w.T}, amortised per token) + "
+        fp4 = " (index keys and queries through RMSNorm / RoPE / Hadamard and FP4)" if self.w.extra.get("fp4_indexer") else ""
+        return (f"full csa_compress of the KV entries and the index keys{fp4} (T={self.w.T}, amortised per token) + "
                 f"indexer over every visible entry, top-{self.w.k} and hybrid attention of {self.n} query tokens "
                 f"({len(self.starts)} groups of {self.G} consecutive tokens evenly spaced over the layer)")
 
@@ -1158,12 +1172,15 @@ def measure(name, args, world, rank, dist, device, torch, C):
 def cpu_baseline(name, w):
     """The oracle on a bounded sample of the workload, on this host's cores (about 10 s)."""
     import oracle as O
-    if name == "hca_prefill_32k":
+    if w.kind == "hca_prefill":
         tps, secs, desc = oracle_hca_sample(w)
-    elif name == "csa_prefill_64k":
+    elif w.kind == "csa_prefill":
         tps, secs, desc = oracle_csa_sample(w)
     else:
-        job_o = OracleDecode(w, 4) if name == "csa_decode_1m" else OracleMixed(w, 8)
+        if w.kind == "csa_decode":
+            job_o = OracleDecode(w, 1 if w.extra.get("shared_prefix") else 4)
+        else:
+            job_o = OracleMixed(w, 8)
         tps, secs, reps = oracle_repeat(job_o)
         desc = f"{job_o.describe()}; the sample timed {reps} times over"
     unit = "tokens/s (sequence x layer)" if w.kind == "mixed_decode" else "tokens/s"

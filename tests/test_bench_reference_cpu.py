@@ -5,6 +5,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -56,3 +57,41 @@ def test_hca_oracle_sample_groups_and_repeat():
             return 8 / 0.25, 0.25
     tps, secs, reps = b.oracle_repeat(Fixed(), target_s=1.0)
     assert reps == 4 and np.isclose(secs, 1.0) and np.isclose(tps, 32.0)
+
+
+def test_cpu_baseline_covers_every_default_workload(monkeypatch):
+    """The default bench line carries a cpu_baseline for every workload it times: the dispatch
+    picks an oracle sample for each workload kind and variant (stubs stand in for the oracle)."""
+    b = _bench()
+    made = []
+
+    class Stub:
+        def __init__(self, w, n_seq=1, seed_rank=0):
+            made.append((w.name if hasattr(w, "name") else w, type(self).__name__, n_seq))
+
+        def describe(self):
+            return "stub"
+
+    monkeypatch.setattr(b, "oracle_hca_sample", lambda w: (1.0, 1.0, "hca"))
+    monkeypatch.setattr(b, "oracle_csa_sample", lambda w: (1.0, 1.0, "csa"))
+    monkeypatch.setattr(b, "oracle_repeat", lambda job: (1.0, 1.0, 1))
+    monkeypatch.setattr(b, "OracleDecode", type("OracleDecode", (Stub,), {}))
+    monkeypatch.setattr(b, "OracleMixed", type("OracleMixed", (Stub,), {}))
+    for name in b.DEFAULT_WORKLOADS:
+        r = b.cpu_baseline(name, b.WL.WORKLOADS[name])
+        assert r["kind"] == "oracle" and r["value"] == 1.0 and r["sample"]
+    kinds = [k for _, k, _ in made]
+    assert kinds.count("OracleDecode") == 2 and kinds.count("OracleMixed") == 1
+    assert sorted(n for _, k, n in made if k == "OracleDecode") == [1, 4]   # shared-prefix decode: 1 sequence x 8 tokens
+
+
+def test_oracle_decode_shared_prefix_tokens():
+    """The shared-prefix decode sample runs G = 8 consecutive tokens of one sequence, positions
+    T-7 .. T, and counts them all."""
+    b = _bench()
+    w = b.WL.WORKLOADS["csa_decode_1m_mtp"]
+    job = b.OracleDecode.__new__(b.OracleDecode)
+    job.w, job.n, job.G = w, 1, 8
+    job.t = np.arange(w.T - 7, w.T + 1)
+    assert list(job.t) == [w.T - 7 + j for j in range(8)]
+    assert "8 new tokens each" in job.describe()
