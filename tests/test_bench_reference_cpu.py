@@ -91,7 +91,7 @@ def test_oracle_decode_shared_prefix_tokens():
     b = _bench()
     w = b.WL.WORKLOADS["csa_decode_1m_mtp"]
     job = b.OracleDecode.__new__(b.OracleDecode)
-    job.w, job.n, job.G = w, 1, 8
+    job.w, job.n, job.G, job.nv = w, 1, 8, (w.T + 1) // w.m
     job.t = np.arange(w.T - 7, w.T + 1)
     assert list(job.t) == [w.T - 7 + j for j in range(8)]
     assert "8 new tokens each" in job.describe()
