@@ -454,6 +454,7 @@ CSA_PATH_PREFILL_TC = 4
 CSA_PATH_PREFILL_GENERIC = 5
 CSA_PATH_DECODE_TC = 6
 CSA_PATH_DECODE_GENERIC = 7
+CSA_PATH_PREFILL_KEYS_TC = 8
 
 
 def csa_set_wait_limit_ns(ns: int) -> int:

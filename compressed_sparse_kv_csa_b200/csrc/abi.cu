@@ -40,7 +40,7 @@ int device_sms()
     return n;
 }
 cudaError_t launch_attn_prefill_generic(const PrefillArgs &a, cudaStream_t st);
-cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled);
+cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled, bool *keys_on_m);
 cudaError_t launch_indexer_scores_tc(const IndexerArgs &a, cudaStream_t st, bool *handled);
 size_t decode_indexer_workspace(int64_t Nq, int64_t max_nvis, int k);
 size_t decode_indexer_need(int64_t Nq, int64_t max_nvis, int k);
@@ -398,10 +398,10 @@ int hybrid_attn_prefill(const void *q, const void *x_win, const void *kv_comp, i
     if (T == 0) return CSA_OK;
     PrefillArgs a{q, x_win, kv_comp, n_comp, idx, idx ? k : 0, sink, scale, T, H, c, m, W, dtype, o, lse,
                   dev_error_word()};
-    bool handled = false;
-    cudaError_t e = launch_attn_prefill_tc(a, S(stream), &handled);
+    bool handled = false, keys_on_m = false;
+    cudaError_t e = launch_attn_prefill_tc(a, S(stream), &handled, &keys_on_m);
     if (handled) {
-        note_path(CSA_PATH_PREFILL_TC);
+        note_path(keys_on_m ? CSA_PATH_PREFILL_KEYS_TC : CSA_PATH_PREFILL_TC);
         return status_of(e);
     }
     note_path(CSA_PATH_PREFILL_GENERIC);

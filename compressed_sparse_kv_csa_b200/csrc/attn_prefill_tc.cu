@@ -443,9 +443,19 @@ bool encode_rows512(CUtensorMap *m, const void *base, uint64_t rows, uint32_t bo
 
 } // namespace
 
-cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled)
+cudaError_t launch_attn_prefill_keys(const PrefillArgs &a, cudaStream_t st, bool *handled);
+
+cudaError_t launch_attn_prefill_tc(const PrefillArgs &a, cudaStream_t st, bool *handled, bool *keys_on_m)
 {
     *handled = false;
+    *keys_on_m = false;
+    if (!a.idx) { // HCA: the kernel with keys on M (measured faster for every-visible-entry layers)
+        cudaError_t e = launch_attn_prefill_keys(a, st, handled);
+        if (*handled) {
+            *keys_on_m = true;
+            return e;
+        }
+    }
     if (a.dtype != CSA_BF16 || a.H != kH || a.c != kC || a.W != kW || a.T <= 0) return cudaSuccess;
     if (a.idx && a.k > 4096) return cudaSuccess;
     if ((uint64_t)a.T * kH >= (1ull << 31)) return cudaSuccess; // TMA row coordinates are int32

@@ -419,6 +419,7 @@ int csa_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int
 #define CSA_PATH_PREFILL_GENERIC 5
 #define CSA_PATH_DECODE_TC 6        /* 64 x 512: tcgen05 split-K attention + merge */
 #define CSA_PATH_DECODE_GENERIC 7
+#define CSA_PATH_PREFILL_KEYS_TC 8   /* bf16 64 x 512, W = 128, HCA: tcgen05 with keys on M (M = 128 MMAs) */
 int32_t csa_last_path(void);
 
 /*

@@ -68,7 +68,7 @@ def test_hca_prefill_32k_full(C):
     np.testing.assert_allclose(host(kv), ref_kv, atol=2e-5, rtol=0)
     # attention: sampled rows; the oracle runs on its own entries stored in bf16, the GPU layer on its
     # own (compression and storage rounding stay inside the 2e-2 tolerance)
-    assert C.csa_last_path() == C.CSA_PATH_PREFILL_TC
+    assert C.csa_last_path() == C.CSA_PATH_PREFILL_KEYS_TC
     rows = _sample_rows(T, m, 11)
     qs = np.stack([WL.draw(w, "q", int(t), int(t) + 1)[0] for t in rows]).reshape(len(rows), H, c)
     kv_store = O.bf16_value(O.bf16_bits(ref_kv))

@@ -390,10 +390,11 @@ def test_prefill_attention_hca_bf16(C, T, W, m):
 @pytest.mark.parametrize("T,m,k", [(1, 4, None), (2, 4, None), (77, 4, None), (130, 128, None), (257, 64, None),
                                    (300, 16, None), (2000, 16, None), (300, 4, 512), (157, 4, 200)])
 def test_prefill_attention_tensor_core_shapes(C, T, m, k):
-    """64 heads x 512 channels, bf16, window 128: the tcgen05 path, one token (64 heads) per pass.
-    HCA (all visible entries): one and two tokens, odd token counts, block boundaries at m = 4, 16,
-    64, 128, fewer tokens than CTAs and several per CTA.  CSA (top-k lists): 4 top-k tiles with
-    many empty (-1) slots and a length that is not a multiple of the 128-key tile."""
+    """64 heads x 512 channels, bf16, window 128: the tcgen05 paths, one token (64 heads) per pass.
+    HCA (all visible entries, the kernel with keys on M): one and two tokens, odd token counts,
+    block boundaries at m = 4, 16, 64, 128, fewer tokens than CTAs and several per CTA.  CSA (top-k
+    lists, the M = 64 kernel): 4 top-k tiles with many empty (-1) slots and a length that is not a
+    multiple of the 128-key tile."""
     w = _wl("csa_prefill_64k", T=T, m=m)
     n_comp = max(T // m, 1)
     q, X, KVc, sink = _prefill_inputs(w, T, n_comp)
@@ -402,7 +403,7 @@ def test_prefill_attention_tensor_core_shapes(C, T, m, k):
     lse = torch.empty((T, 64), dtype=torch.float32, device="cuda")
     o = C.hybrid_attn_prefill(dev(q, "bf16"), dev(X, "bf16"), dev(KVc, "bf16"), dev(sink), 1.0, m, 128,
                               idx=None if idx is None else dev_i(idx), lse=lse)
-    assert C.csa_last_path() == C.CSA_PATH_PREFILL_TC
+    assert C.csa_last_path() == (C.CSA_PATH_PREFILL_KEYS_TC if k is None else C.CSA_PATH_PREFILL_TC)
     err = row_rel_err(host(o), o_ref)
     assert err.max() < 2e-2, err.max()
     np.testing.assert_allclose(host(lse), lse_ref, atol=2e-3)
