@@ -232,6 +232,8 @@ int csa_prep_rows(const void *x, int32_t in_dtype, int64_t n, int32_t d, const f
  *   w        [Nq, H_I] fp32 head weights (any scaling already folded in by the caller)
  *   q_pos    [Nq] int64 absolute 0-based positions, or NULL for q_pos[r] = r (prefill)
  *   key_off  [Nq] int64 first key row of each query's sequence, or NULL for all 0
+ *            (FP4 keys: sequences that start at a multiple of 4 rows, in a cache of a multiple of
+ *            4 rows, take the faster tile path; any start is correct)
  *   max_nvis host-side upper bound of nv(r) (sizes the score buffer)
  *   idx_out  [Nq, k] int32;  score_out [Nq, k] fp32 scores of the selected entries (or NULL;
  *            -inf in padded slots)
