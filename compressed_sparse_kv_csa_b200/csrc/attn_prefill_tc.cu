@@ -354,7 +354,6 @@ __device__ __forceinline__ bool mma_role(const PrefillArgs &a, const Smem &S, ui
     uint32_t q_ph = 0, kf_ph[2] = {0, 0}, p_ph = 0;
     for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
         const int64_t n_cmp = n_compressed(a, t);
-        const int64_t nvt = (t + 1) / a.m; // N_vis(t), once per token
         const int nt = n_tiles(n_cmp);
         if (!mbar_wait(S.bar(B_QFULL), q_ph)) return false;
         q_ph ^= 1;
