@@ -20,11 +20,13 @@
 //     B = P^T [64 heads x 128 keys] (K-major); M=128, N=64, K=128.  O^T of quarter c at columns
 //     64c .. 64c+63, TMEM lane = channel 128c + lane; the whole 512 x 64 fp32 output stays in TMEM
 //     for the token's key loop.
-//   * Softmax over the keys = across TMEM lanes.  Thread (warp w, lane l) holds key 32w+l's 64
-//     head scores.  Per-head maxima and sums go by a warp reduce-scatter (five shuffle rounds that
-//     halve the heads each time, leaving heads 2l, 2l+1 on lane l) and across the four warps by
-//     shared memory.  Online softmax in the log2 domain with a lazy rescale: a head's running max
-//     moves (and its O^T column is rescaled in TMEM) only when a tile raises it by more than 8.
+//   * Softmax over the keys = across TMEM lanes.  Eight warps: warps w and w+4 reach the lanes of
+//     keys 32(w%4) .. 32(w%4)+31 and take heads 0-31 and 32-63 of them.  Per-head maxima go
+//     through bf16 copies of the scores in the P^T buffer (four threads per head row, with a
+//     margin for the copy's rounding); per-head sums in fp32 by a warp reduce-scatter, added
+//     across the lane quarters at the end of the token.  Online softmax in the log2 domain with a
+//     lazy rescale: a head's running max moves (and its O^T column is rescaled in TMEM) only when
+//     a tile raises it by more than 8.
 //   * The key tile arrives in four channel quarters; quarter c is released as soon as the O^T MMAs
 //     of quarter c complete, so the next tile's loads overlap the rest of P V.
 //   * Keys per token: tile 0 = window rows t-127..t of x_win; then tiles of 128 compressed rows
