@@ -417,7 +417,7 @@ int csa_decode_glue(const void *o, const void *P, const void *Rm, int64_t R, int
 #define CSA_PATH_INDEXER_FP4_TC 1   /* FP4 64 x 128: tcgen05 kind::mxf4 scan + threshold merge */
 #define CSA_PATH_INDEXER_BF16_TC 2  /* bf16 64 x 128 prefill: tcgen05 scores + per-query top-k */
 #define CSA_PATH_INDEXER_GENERIC 3  /* any other shape: CUDA-core scores + per-query top-k */
-#define CSA_PATH_PREFILL_TC 4       /* bf16 64 x 512, W = 128: tcgen05 attention */
+#define CSA_PATH_PREFILL_TC 4       /* bf16 64 x 512, W = 128, CSA (top-k lists): tcgen05, one token on M = 64 */
 #define CSA_PATH_PREFILL_GENERIC 5
 #define CSA_PATH_DECODE_TC 6        /* 64 x 512: tcgen05 split-K attention + merge */
 #define CSA_PATH_DECODE_GENERIC 7

@@ -44,6 +44,17 @@ def test_library_exports_every_declared_symbol(C):
         assert hasattr(C.lib(), n)
 
 
+def test_binding_mirrors_every_header_constant(C):
+    """Every integer #define CSA_* of include/csa.h (status codes, device error bits, path codes,
+    dtypes) has the same value in the Python binding."""
+    src = open(os.path.join(ROOT, "include", "csa.h")).read()
+    defs = dict(re.findall(r"^#define\s+(CSA_[A-Z0-9_]+)\s+\(?(-?(?:0x[0-9a-fA-F]+|\d+))u?\)?", src, flags=re.M))
+    assert len(defs) >= 20 and "CSA_PATH_PREFILL_KEYS_TC" in defs
+    for name, v in defs.items():
+        assert hasattr(C, name), name
+        assert getattr(C, name) == int(v, 0), (name, getattr(C, name), v)
+
+
 def test_status_strings_and_version(C):
     assert C.csa_abi_version() == 101
     assert C.status_string(0) == "ok"
