@@ -167,3 +167,51 @@ def test_paged_decode_reads_equal_contiguous_reads(C):
     torch.cuda.synchronize()
     assert C.csa_device_error() == 0
     assert torch.equal(o1, o2) and torch.equal(o3, o4)
+
+
+@pytest.mark.parametrize("page_rows", [8, 64, 128])
+def test_paged_fp4_scan_page_sizes(C, page_rows):
+    """The FP4 scan over paged keys for other page sizes: 64- and 128-row pages take the permuted
+    tiles (one box per page and residue), 8-row pages the natural order; both equal the scan of
+    the same keys stored contiguously, indices and scores bit for bit."""
+    w = WL.WORKLOADS["csa_decode_1m"]
+    Bn, k, Hi, d, m = 3, 256, 64, 128, 4
+    g = np.random.default_rng(page_rows)
+    pos = np.array([4 * 5000 + 1, 4 * 1234 + 3, 4 * 300], np.int64)
+    nv = O.n_vis(pos, m)
+    off = np.concatenate([[0], np.cumsum(nv)[:-1]]).astype(np.int64)
+    n_pages = -(-nv // page_rows)
+    max_pages = int(n_pages.max())
+    pool_pages = int(n_pages.sum()) + 2
+    perm = g.permutation(pool_pages)
+    pages = np.full((Bn, max_pages), -1, np.int32)
+    used = 0
+    for b in range(Bn):
+        pages[b, :n_pages[b]] = perm[used:used + n_pages[b]]
+        used += n_pages[b]
+    keys = np.concatenate([WL.draw(w, "KI", 0, int(n), seq=95 + b) for b, n in enumerate(nv)])
+    k4 = C.Fp4Rows.empty(len(keys), d, "cuda")
+    C.csa_quantize_fp4(dev(keys), k4)
+    prow = np.concatenate([pages[b, np.arange(nv[b]) // page_rows].astype(np.int64) * page_rows
+                           + np.arange(nv[b]) % page_rows for b in range(Bn)])
+    pr = torch.from_numpy(prow).cuda()
+    pk4 = C.Fp4Rows.empty(pool_pages * page_rows, d, "cuda")
+    pk4.codes.zero_()
+    pk4.scales.zero_()
+    pk4.codes[pr] = k4.codes
+    pk4.scales[pr] = k4.scales
+    qx = np.stack([WL.draw(w, "qI", 0, 1, seq=95 + b).reshape(Hi, d) for b in range(Bn)])
+    q4 = C.Fp4Rows.empty(Bn * Hi, d, "cuda")
+    C.csa_quantize_fp4(dev(qx.reshape(Bn * Hi, d)), q4)
+    wt = dev(np.concatenate([WL.draw(w, "w", 0, 1, seq=95 + b) for b in range(Bn)]))
+    pos_d = torch.from_numpy(pos).cuda()
+    sc1 = torch.empty((Bn, k), dtype=torch.float32, device="cuda")
+    sc2 = torch.empty_like(sc1)
+    i1 = C.indexer_topk(q4, wt, k4, m, k, max_nvis=int(nv.max()), q_pos=pos_d, key_off=torch.from_numpy(off).cuda(),
+                        score_out=sc1)
+    i2 = C.indexer_topk_paged(q4, wt, pk4, m, k, max_nvis=int(nv.max()), pages=torch.from_numpy(pages).cuda(),
+                              page_rows=page_rows, q_pos=pos_d, score_out=sc2)
+    assert C.csa_last_path() == C.CSA_PATH_INDEXER_FP4_TC
+    torch.cuda.synchronize()
+    assert C.csa_device_error() == 0
+    assert torch.equal(i1, i2) and torch.equal(sc1, sc2)
